@@ -1,0 +1,258 @@
+/*
+ * Plain fp64 reference for paged-KV decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the oracle that the CUDA library is
+ * checked against. Only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg may load it; the product path never does. It shares no
+ * code, header, table or constant with the CUDA library.
+ *
+ * What it computes (single-threaded, double precision, no blocking, no
+ * online rescaling, no split): for every sequence b, query row i and query
+ * head h, plain softmax attention over the keys the row may see, walking the
+ * page table one token at a time.
+ *
+ * Sources, by page and section:
+ *  - "AstrAI commit log, attn_paged_decode_split_kv_mma.cuh": the scalar
+ *    variant resolves the page table per position when it loads K/V; the
+ *    split-KV partials are later combined; causal_offset semantics
+ *    (-1 = off, >= 0 = position of the first query row).
+ *  - "b12x 0.30.0, Kernel inventory, Attention table, Paged attention row":
+ *    bf16 and FP8-E4M3 KV caches, sliding window, GQA, split-KV or direct
+ *    output, persistent merge kernel.
+ *  - "sglang profiler skill, fuse-overlap catalog, vLLM-origin attention +
+ *    output quant row": merge_attn_states combines attention states by their
+ *    log-sum-exp.
+ *
+ * Readings taken where the pages are silent:
+ *  R1 lse is the natural log of sum_j exp(scale * q.k_j).
+ *  R2 causal_offset = -2 means bottom-right alignment: pos_i = L_b - q_len + i.
+ *  R3 a window of W keys includes the query's own position:
+ *     visible iff j >= pos_i - W + 1; W <= 0 is off; with causal off the
+ *     window is measured from L_b - 1.
+ *  R4 GQA head mapping is consecutive: kv head = h / (Hq / Hkv).
+ *  R5 KV pool layout is [num_pages, Hkv, page_size, D].
+ *  R6 FP8 value = decode_e4m3(byte) * kv_scale, one scale for K and V.
+ *  R8 a row that sees no key has out = 0 and lse = -inf.
+ *
+ * Pins (tests/test_oracle.py): brute-force dense attention over the unpaged
+ * K/V, page-permutation invariance, split-merge invariance, closed forms
+ * (equal keys -> mean of V, one key -> v, one-hot V -> probabilities),
+ * e4m3/bf16 decode against torch's independent float8/bfloat16 casts, and
+ * hand-derived golden fixtures.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fPIC -shared oracle.c -o liboracle.so -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Status codes returned by the oracle. */
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_BAD_PAGE 2
+#define ORACLE_NO_MEMORY 3
+
+#define ORACLE_KV_BF16 0
+#define ORACLE_KV_FP8_E4M3 1
+
+#define ORACLE_CAUSAL_OFF (-1)
+#define ORACLE_CAUSAL_BOTTOM_RIGHT (-2)
+
+/* bf16 is the upper half of an IEEE binary32: widen by a 16-bit shift. */
+double oracle_bf16_to_double(uint16_t bits) {
+  uint32_t u = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* FP8 E4M3 ("fn" variant, no infinities) from its fields:
+ * sign bit, 4 exponent bits with bias 7, 3 mantissa bits.
+ * exponent 0 is subnormal: m/8 * 2^(1-7); S.1111.111 is NaN;
+ * every other code is (1 + m/8) * 2^(e-7). Largest finite value 448. */
+double oracle_e4m3_to_double(uint8_t code) {
+  int s = (code >> 7) & 1;
+  int e = (code >> 3) & 0xF;
+  int m = code & 0x7;
+  double mag;
+  if (e == 0xF && m == 0x7) return NAN;
+  if (e == 0)
+    mag = ldexp((double)m / 8.0, 1 - 7);
+  else
+    mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+/* One K or V element of the pool, decoded to double. */
+static double kv_elem(const void* pool, int kv_dtype, double kv_scale,
+                      int64_t index) {
+  if (kv_dtype == ORACLE_KV_BF16)
+    return oracle_bf16_to_double(((const uint16_t*)pool)[index]);
+  return oracle_e4m3_to_double(((const uint8_t*)pool)[index]) * kv_scale;
+}
+
+/* Position of query row i of sequence b (reading R2/R3). */
+static int64_t row_position(int causal_offset, int64_t kv_len, int q_len,
+                            int i) {
+  if (causal_offset >= 0) return (int64_t)causal_offset + i;
+  if (causal_offset == ORACLE_CAUSAL_BOTTOM_RIGHT)
+    return kv_len - (int64_t)q_len + i;
+  return kv_len - 1; /* causal off: only the window uses it */
+}
+
+/* Is logical key j visible to a query row at position pos? */
+static int key_visible(int64_t j, int64_t kv_len, int causal, int64_t pos,
+                       int window) {
+  if (j < 0 || j >= kv_len) return 0;
+  if (causal && j > pos) return 0;
+  if (window > 0 && j < pos - (int64_t)window + 1) return 0;
+  return 1;
+}
+
+/*
+ * out[b, i, h, :] and lse[b, i, h] for every row, restricted to keys in
+ * [tok_lo, tok_hi) (tok_hi < 0 means no restriction). The restriction lets
+ * the tests build split partials from the same definition.
+ *
+ * q          bf16 bits  [B, q_len, Hq, D]
+ * k/v_pages  bf16 bits or e4m3 bytes  [num_pages, Hkv, page_size, D]
+ * page_table int32 [B, max_pages]; kv_lens int32 [B]
+ * out        double [B, q_len, Hq, D]; lse double [B, q_len, Hq]
+ */
+int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
+                             const void* v_pages, const int32_t* page_table,
+                             const int32_t* kv_lens, int B, int q_len, int Hq,
+                             int Hkv, int D, int page_size, int max_pages,
+                             int num_pages, float scale, int causal_offset,
+                             int window, int kv_dtype, float kv_scale,
+                             int64_t tok_lo, int64_t tok_hi, double* out,
+                             double* lse) {
+  if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || D < 1 || page_size < 1 ||
+      max_pages < 0 || num_pages < 0 || Hq % Hkv != 0)
+    return ORACLE_BAD_ARG;
+  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3)
+    return ORACLE_BAD_ARG;
+  if (causal_offset < ORACLE_CAUSAL_BOTTOM_RIGHT) return ORACLE_BAD_ARG;
+
+  const int G = Hq / Hkv;
+  const int causal = causal_offset != ORACLE_CAUSAL_OFF;
+  const double dscale = (double)scale;
+  const double dkv_scale = (double)kv_scale;
+
+  int64_t max_len = 0;
+  for (int b = 0; b < B; ++b) {
+    if (kv_lens[b] < 0) return ORACLE_BAD_ARG;
+    if (kv_lens[b] > (int64_t)max_pages * page_size) return ORACLE_BAD_ARG;
+    if (kv_lens[b] > max_len) max_len = kv_lens[b];
+  }
+  double* s = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+  if (!s) return ORACLE_NO_MEMORY;
+
+  for (int b = 0; b < B; ++b) {
+    const int64_t L = kv_lens[b];
+    for (int i = 0; i < q_len; ++i) {
+      const int64_t pos = row_position(causal_offset, L, q_len, i);
+      for (int h = 0; h < Hq; ++h) {
+        const int g = h / G; /* reading R4 */
+        const uint16_t* qrow = q + (((int64_t)b * q_len + i) * Hq + h) * D;
+        double* orow = out + (((int64_t)b * q_len + i) * Hq + h) * D;
+        double* lrow = lse + ((int64_t)b * q_len + i) * Hq + h;
+
+        /* Pass 1: scores of the visible keys, walking the page table. */
+        double m = -INFINITY;
+        int64_t nvis = 0;
+        for (int64_t j = 0; j < L; ++j) {
+          int vis = key_visible(j, L, causal, pos, window);
+          if (vis && tok_hi >= 0 && (j < tok_lo || j >= tok_hi)) vis = 0;
+          if (!vis) {
+            s[j] = -INFINITY;
+            continue;
+          }
+          const int32_t page = page_table[(int64_t)b * max_pages + j / page_size];
+          if (page < 0 || page >= num_pages) {
+            free(s);
+            return ORACLE_BAD_PAGE;
+          }
+          const int64_t row = j % page_size;
+          const int64_t base = (((int64_t)page * Hkv + g) * page_size + row) * D;
+          double dot = 0.0;
+          for (int d = 0; d < D; ++d)
+            dot += oracle_bf16_to_double(qrow[d]) *
+                   kv_elem(k_pages, kv_dtype, dkv_scale, base + d);
+          s[j] = dscale * dot;
+          if (s[j] > m) m = s[j];
+          ++nvis;
+        }
+
+        if (nvis == 0) { /* reading R8 */
+          for (int d = 0; d < D; ++d) orow[d] = 0.0;
+          *lrow = -INFINITY;
+          continue;
+        }
+
+        /* lse = m + ln sum_j exp(s_j - m)  (reading R1) */
+        double sum = 0.0;
+        for (int64_t j = 0; j < L; ++j)
+          if (s[j] != -INFINITY) sum += exp(s[j] - m);
+        const double row_lse = m + log(sum);
+        *lrow = row_lse;
+
+        /* Pass 2: out = sum_j exp(s_j - lse) * v_j. */
+        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+          if (s[j] == -INFINITY) continue;
+          const double p = exp(s[j] - row_lse);
+          const int32_t page = page_table[(int64_t)b * max_pages + j / page_size];
+          const int64_t row = j % page_size;
+          const int64_t base = (((int64_t)page * Hkv + g) * page_size + row) * D;
+          for (int d = 0; d < D; ++d)
+            orow[d] += p * kv_elem(v_pages, kv_dtype, dkv_scale, base + d);
+        }
+      }
+    }
+  }
+  free(s);
+  return ORACLE_OK;
+}
+
+/*
+ * Log-sum-exp merge of n attention states over disjoint key sets
+ * (merge_attn_states / PagedPersistentMergeKernel):
+ *   lse = m* + ln sum_s exp(lse_s - m*),  m* = max_s lse_s
+ *   out = sum_s exp(lse_s - lse) * out_s
+ * All states empty (every lse_s = -inf): out = 0, lse = -inf.
+ *
+ * o_parts [n, rows, D], lse_parts [n, rows]; out [rows, D], lse [rows].
+ */
+int oracle_merge_states(const double* o_parts, const double* lse_parts, int n,
+                        int64_t rows, int D, double* out, double* lse) {
+  if (n < 1 || rows < 0 || D < 1) return ORACLE_BAD_ARG;
+  for (int64_t r = 0; r < rows; ++r) {
+    double m = -INFINITY;
+    for (int s = 0; s < n; ++s)
+      if (lse_parts[(int64_t)s * rows + r] > m) m = lse_parts[(int64_t)s * rows + r];
+    double* orow = out + r * D;
+    if (m == -INFINITY) {
+      for (int d = 0; d < D; ++d) orow[d] = 0.0;
+      lse[r] = -INFINITY;
+      continue;
+    }
+    double sum = 0.0;
+    for (int s = 0; s < n; ++s) {
+      const double ls = lse_parts[(int64_t)s * rows + r];
+      if (ls != -INFINITY) sum += exp(ls - m);
+    }
+    const double total = m + log(sum);
+    lse[r] = total;
+    for (int d = 0; d < D; ++d) orow[d] = 0.0;
+    for (int s = 0; s < n; ++s) {
+      const double ls = lse_parts[(int64_t)s * rows + r];
+      if (ls == -INFINITY) continue;
+      const double w = exp(ls - total);
+      const double* op = o_parts + ((int64_t)s * rows + r) * D;
+      for (int d = 0; d < D; ++d) orow[d] += w * op[d];
+    }
+  }
+  return ORACLE_OK;
+}

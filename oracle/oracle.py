@@ -1,0 +1,144 @@
+"""ctypes wrapper around ``oracle.c`` (test infrastructure only).
+
+The C file is the oracle: plain single-threaded fp64 softmax attention that
+walks the page table token by token. This module only builds it, loads it and
+marshals numpy arrays in and out; it holds none of the method's arithmetic.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+ORACLE_KV_BF16 = 0
+ORACLE_KV_FP8_E4M3 = 1
+CAUSAL_OFF = -1
+CAUSAL_BOTTOM_RIGHT = -2
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(out_path: str = _LIB_PATH, extra_flags=()) -> str:
+    """Compile oracle.c into a shared library with gcc and return its path.
+
+    ``-ffp-contract=off`` keeps every multiply and add a separately rounded
+    IEEE double operation.
+    """
+    cmd = [
+        "gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-Wall",
+        *extra_flags, _SRC, "-o", out_path, "-lm",
+    ]
+    subprocess.run(cmd, check=True)
+    return out_path
+
+
+def _needs_build() -> bool:
+    if not os.path.exists(_LIB_PATH):
+        return True
+    return os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+
+
+def load(path: str | None = None):
+    """Load (building first if stale) the oracle shared library."""
+    global _lib
+    if path is not None:
+        return _declare(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            if _needs_build():
+                build()
+            _lib = _declare(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def _declare(lib):
+    lib.oracle_bf16_to_double.restype = ctypes.c_double
+    lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+    lib.oracle_e4m3_to_double.restype = ctypes.c_double
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    p = ctypes.c_void_p
+    i32 = ctypes.c_int
+    lib.oracle_paged_decode_attn.restype = i32
+    lib.oracle_paged_decode_attn.argtypes = [
+        p, p, p, p, p,                      # q, k, v, page_table, kv_lens
+        i32, i32, i32, i32, i32, i32, i32, i32,  # B Lq Hq Hkv D P max_pages num_pages
+        ctypes.c_float, i32, i32, i32, ctypes.c_float,  # scale causal window dtype kv_scale
+        ctypes.c_int64, ctypes.c_int64,     # tok_lo, tok_hi
+        p, p,                               # out, lse
+    ]
+    lib.oracle_merge_states.restype = i32
+    lib.oracle_merge_states.argtypes = [p, p, i32, ctypes.c_int64, i32, p, p]
+    return lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def bf16_to_double(bits: int, lib=None) -> float:
+    return (lib or load()).oracle_bf16_to_double(int(bits))
+
+
+def e4m3_to_double(code: int, lib=None) -> float:
+    return (lib or load()).oracle_e4m3_to_double(int(code))
+
+
+def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
+                      num_kv_heads, page_size, scale, causal_offset=CAUSAL_OFF,
+                      window=0, kv_dtype=ORACLE_KV_BF16, kv_scale=1.0,
+                      tok_range=None, lib=None):
+    """Run the oracle on host arrays.
+
+    q_bits      uint16 [B, q_len, Hq, D]   (bf16 bit patterns)
+    k/v_pages   uint16 or uint8 [num_pages, Hkv, page_size, D]
+    page_table  int32 [B, max_pages];  kv_lens int32 [B]
+    tok_range   optional (lo, hi): keep only keys with lo <= j < hi
+    Returns (out float64 [B, q_len, Hq, D], lse float64 [B, q_len, Hq]).
+    """
+    lib = lib or load()
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kdt = np.uint16 if kv_dtype == ORACLE_KV_BF16 else np.uint8
+    k_pages = np.ascontiguousarray(k_pages, dtype=kdt)
+    v_pages = np.ascontiguousarray(v_pages, dtype=kdt)
+    page_table = np.ascontiguousarray(page_table, dtype=np.int32)
+    kv_lens = np.ascontiguousarray(kv_lens, dtype=np.int32)
+    B, q_len, Hq, D = q_bits.shape
+    num_pages = k_pages.shape[0]
+    assert k_pages.shape == v_pages.shape
+    assert k_pages.shape[1:] == (num_kv_heads, page_size, D), k_pages.shape
+    max_pages = page_table.shape[1] if page_table.ndim == 2 else 0
+    out = np.zeros((B, q_len, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, q_len, Hq), dtype=np.float64)
+    lo, hi = (0, -1) if tok_range is None else tok_range
+    rc = lib.oracle_paged_decode_attn(
+        _ptr(q_bits), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+        _ptr(kv_lens), B, q_len, Hq, num_kv_heads, D, page_size, max_pages,
+        num_pages, float(scale), int(causal_offset), int(window),
+        int(kv_dtype), float(kv_scale), int(lo), int(hi), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_decode_attn failed with status {rc}")
+    return out, lse
+
+
+def merge_states(o_parts, lse_parts, lib=None):
+    """LSE merge of n states: o_parts [n, rows, D], lse_parts [n, rows]."""
+    lib = lib or load()
+    o_parts = np.ascontiguousarray(o_parts, dtype=np.float64)
+    lse_parts = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    n, rows, D = o_parts.shape
+    out = np.zeros((rows, D), dtype=np.float64)
+    lse = np.zeros((rows,), dtype=np.float64)
+    rc = lib.oracle_merge_states(_ptr(o_parts), _ptr(lse_parts), n, rows, D,
+                                 _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_merge_states failed with status {rc}")
+    return out, lse

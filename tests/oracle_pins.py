@@ -1,0 +1,325 @@
+"""Checks that pin the fp64 oracle to things other than itself.
+
+Each check takes the loaded oracle library as an argument, so the same checks
+run against the real oracle (tests/test_oracle.py) and against copies of it
+with a planted mistake (which must fail at least one check).
+
+What pins what:
+  * decode_bf16 / decode_e4m3: torch's own bfloat16 and float8_e4m3fn casts
+    (an independent implementation) plus hand-worked E4M3 code values.
+  * bruteforce: textbook dense attention (numpy matmul + scipy logsumexp)
+    over the per-sequence K/V drawn BEFORE they were scattered into pages,
+    so it never touches the page table; visibility is built as a dense
+    boolean matrix rather than the oracle's per-key test.
+  * page_permutation: relabelling physical pages changes nothing, bit for bit.
+  * split_merge: partial states over disjoint key ranges, LSE-merged, equal
+    the unsplit result.
+  * closed forms: equal keys -> mean of visible V and lse = s + ln |V|;
+    one-hot V -> softmax probabilities; single key -> v.
+  * golden: hand-derived fixtures under tests/golden/.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+from scipy.special import logsumexp, softmax
+
+from oracle import oracle as orc
+from paged_kv_decode_30_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+# Small cases: (name, Workload). All use the dense route so that the
+# brute force has an unpaged copy of K/V.
+SMALL_CASES = [
+    W.TINY,
+    W.Workload(name="gqa2_d32_p8", batch=3, num_q_heads=8, num_kv_heads=2,
+               head_dim=32, page_size=8, kv_lens=("fixed", [1, 17, 64]),
+               extra_pages=3, route="dense", seed=11),
+    W.Workload(name="verify3_d16_p4", batch=2, q_len=3, num_q_heads=6,
+               num_kv_heads=3, head_dim=16, page_size=4,
+               causal_offset=W.CAUSAL_BOTTOM_RIGHT, kv_lens=("fixed", [9, 30]),
+               route="dense", seed=12),
+    W.Workload(name="verify4_window16", batch=2, q_len=4, num_q_heads=4,
+               num_kv_heads=2, head_dim=16, page_size=8,
+               causal_offset=W.CAUSAL_BOTTOM_RIGHT, window=16,
+               kv_lens=("fixed", [50, 120]), route="dense",
+               poison_invisible=True, seed=13),
+    W.Workload(name="fixed_offset3", batch=2, q_len=2, num_q_heads=2,
+               num_kv_heads=1, head_dim=8, page_size=16, causal_offset=3,
+               kv_lens=("fixed", [40, 5]), route="dense", seed=14),
+    W.Workload(name="window20_noncausal", batch=2, num_q_heads=4,
+               num_kv_heads=2, head_dim=16, page_size=8, window=20,
+               kv_lens=("fixed", [70, 33]), route="dense",
+               poison_invisible=True, seed=15),
+    W.Workload(name="fp8_verify4_window64", batch=2, q_len=4, num_q_heads=8,
+               num_kv_heads=2, head_dim=32, page_size=16,
+               kv_dtype=W.KV_FP8_E4M3, causal_offset=W.CAUSAL_BOTTOM_RIGHT,
+               window=64, kv_lens=("fixed", [100, 300]), route="dense",
+               poison_invisible=True, seed=16),
+    W.Workload(name="empty_rows", batch=3, num_q_heads=4, num_kv_heads=4,
+               head_dim=16, page_size=4, kv_lens=("fixed", [0, 10, 0]),
+               extra_pages=2, route="dense", seed=17),
+    W.Workload(name="peaked_d64_p32", batch=2, num_q_heads=4, num_kv_heads=1,
+               head_dim=64, page_size=32, kv_lens=("fixed", [256, 130]),
+               peaked_frac=0.05, route="dense", seed=18),
+]
+
+
+def run_oracle(inp, lib, tok_range=None, **over):
+    wl = inp["workload"]
+    kw = dict(num_kv_heads=wl.num_kv_heads, page_size=wl.page_size,
+              scale=W.scale_of(wl), causal_offset=wl.causal_offset,
+              window=wl.window, kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"],
+              tok_range=tok_range)
+    kw.update(over)
+    return orc.paged_decode_attn(
+        W.to_bits(inp["q"]), W.to_bits(inp["k_pages"]), W.to_bits(inp["v_pages"]),
+        inp["page_table"].cpu().numpy(), inp["kv_lens"].cpu().numpy(), lib=lib, **kw)
+
+
+def decode_dense(x: torch.Tensor, kv_dtype: int, kv_scale: float) -> np.ndarray:
+    """Values of a bf16 / e4m3-code tensor as float64, through torch's casts."""
+    if kv_dtype == W.KV_BF16:
+        return x.to(torch.float64).numpy()
+    return x.view(torch.float8_e4m3fn).to(torch.float64).numpy() * kv_scale
+
+
+def visibility_matrix(L, q_len, causal_offset, window):
+    """[q_len, L] boolean: may row i see key j. Dense restatement of the
+    readings (bottom-right / fixed-offset causal, window including the query)."""
+    j = np.arange(L)[None, :]
+    i = np.arange(q_len)[:, None]
+    if causal_offset >= 0:
+        pos = causal_offset + i
+    elif causal_offset == W.CAUSAL_BOTTOM_RIGHT:
+        pos = L - q_len + i
+    else:
+        pos = np.full_like(i, L - 1)
+    vis = np.ones((q_len, L), dtype=bool)
+    if causal_offset != W.CAUSAL_OFF:
+        vis &= j <= pos
+    if window > 0:
+        vis &= j >= pos - window + 1
+    return vis
+
+
+def bruteforce(inp):
+    """Textbook dense softmax attention over the unpaged K/V copies."""
+    wl = inp["workload"]
+    B, Lq, Hq, D = inp["q"].shape
+    G = wl.group
+    scale = W.scale_of(wl)
+    q = inp["q"].to(torch.float64).numpy()
+    out = np.zeros((B, Lq, Hq, D))
+    lse = np.full((B, Lq, Hq), -np.inf)
+    for b in range(B):
+        K = decode_dense(inp["k_dense"][b], wl.kv_dtype, inp["kv_scale"])  # [Hkv, L, D]
+        V = decode_dense(inp["v_dense"][b], wl.kv_dtype, inp["kv_scale"])
+        L = K.shape[1]
+        vis = visibility_matrix(L, Lq, wl.causal_offset, wl.window)
+        for i in range(Lq):
+            sel = vis[i]
+            if not sel.any():
+                continue
+            for h in range(Hq):
+                g = h // G
+                s = scale * (K[g][sel] @ q[b, i, h])
+                lse[b, i, h] = logsumexp(s)
+                out[b, i, h] = np.exp(s - lse[b, i, h]) @ V[g][sel]
+    return out, lse
+
+
+def assert_close(a, b, tol, what):
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    err = np.where(both_inf, 0.0, np.abs(a - b))
+    assert not np.isnan(err).any(), f"{what}: NaN mismatch"
+    m = float(err.max()) if err.size else 0.0
+    assert m <= tol, f"{what}: max abs err {m:.3e} > {tol:.1e}"
+
+
+# --------------------------------------------------------------------------
+# individual checks
+
+
+def check_decode_bf16(lib):
+    bits = np.arange(65536, dtype=np.uint32)
+    ref = torch.from_numpy(bits.astype(np.int32)).to(torch.int16).view(torch.bfloat16)
+    ref = ref.to(torch.float64).numpy()
+    got = np.array([orc.bf16_to_double(int(b), lib=lib) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "bf16 NaN set differs"
+    assert np.array_equal(got[~nan], ref[~nan]), "bf16 decode differs from torch"
+
+
+def check_decode_e4m3(lib):
+    codes = np.arange(256, dtype=np.int32)
+    ref = torch.from_numpy(codes).to(torch.uint8).view(torch.float8_e4m3fn)
+    ref = ref.to(torch.float64).numpy()
+    got = np.array([orc.e4m3_to_double(int(c), lib=lib) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "e4m3 NaN set differs"
+    assert np.array_equal(got[~nan], ref[~nan]), "e4m3 decode differs from torch"
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+    with open(os.path.join(GOLDEN, "e4m3_codes.json")) as f:
+        g = json.load(f)
+    for c, v in zip(g["codes"], g["values"]):
+        x = orc.e4m3_to_double(c, lib=lib)
+        if v == "nan":
+            assert math.isnan(x), hex(c)
+        else:
+            assert x == v and math.copysign(1, x) == math.copysign(1, v), (hex(c), x, v)
+
+
+def check_bruteforce(wl, lib, tol=1e-12):
+    inp = W.generate(wl)
+    out, lse = run_oracle(inp, lib)
+    ref_out, ref_lse = bruteforce(inp)
+    assert_close(out, ref_out, tol, f"{wl.name} out vs brute force")
+    assert_close(lse, ref_lse, tol, f"{wl.name} lse vs brute force")
+
+
+def check_page_permutation(wl, lib, seed=99):
+    inp = W.generate(wl)
+    out0, lse0 = run_oracle(inp, lib)
+    n = inp["k_pages"].shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(seed))
+    k2 = torch.empty_like(inp["k_pages"])
+    v2 = torch.empty_like(inp["v_pages"])
+    k2[perm] = inp["k_pages"]
+    v2[perm] = inp["v_pages"]
+    pt = inp["page_table"].clone().to(torch.int64)
+    pt = torch.where(pt >= 0, perm[pt.clamp(min=0)], pt).to(torch.int32)
+    inp2 = dict(inp, k_pages=k2, v_pages=v2, page_table=pt)
+    out1, lse1 = run_oracle(inp2, lib)
+    assert np.array_equal(out0, out1) and np.array_equal(lse0, lse1), \
+        f"{wl.name}: page permutation changed the result"
+
+
+def check_split_merge(wl, cuts, lib, tol=1e-12):
+    inp = W.generate(wl)
+    out, lse = run_oracle(inp, lib)
+    bounds = [0, *cuts, 1 << 40]
+    parts = [run_oracle(inp, lib, tok_range=(a, b)) for a, b in zip(bounds, bounds[1:])]
+    B, Lq, Hq, D = out.shape
+    o_parts = np.stack([p[0].reshape(-1, D) for p in parts])
+    l_parts = np.stack([p[1].reshape(-1) for p in parts])
+    mo, ml = orc.merge_states(o_parts, l_parts, lib=lib)
+    assert_close(mo, out.reshape(-1, D), tol, f"{wl.name} split {cuts} out")
+    assert_close(ml, lse.reshape(-1), tol, f"{wl.name} split {cuts} lse")
+
+
+def check_equal_keys(lib, tol=1e-12):
+    """All keys equal -> out = mean of the visible v, lse = s + ln |visible|."""
+    wl = W.Workload(name="equal_keys", batch=2, q_len=3, num_q_heads=4,
+                    num_kv_heads=2, head_dim=16, page_size=8,
+                    causal_offset=W.CAUSAL_BOTTOM_RIGHT, window=20,
+                    kv_lens=("fixed", [45, 7]), route="dense", seed=21)
+    inp = W.generate(wl)
+    kvec = torch.randn(wl.head_dim, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    valid = ~torch.isnan(inp["k_pages"].float())
+    inp["k_pages"] = torch.where(valid, kvec.expand_as(inp["k_pages"]), inp["k_pages"])
+    out, lse = run_oracle(inp, lib)
+    q = inp["q"].to(torch.float64).numpy()
+    k = kvec.to(torch.float64).numpy()
+    scale = W.scale_of(wl)
+    for b in range(wl.batch):
+        V = inp["v_dense"][b].to(torch.float64).numpy()
+        L = V.shape[1]
+        vis = visibility_matrix(L, wl.q_len, wl.causal_offset, wl.window)
+        for i in range(wl.q_len):
+            n = int(vis[i].sum())
+            for h in range(wl.num_q_heads):
+                g = h // wl.group
+                assert_close(out[b, i, h], V[g][vis[i]].mean(axis=0), tol, "equal keys mean")
+                s = scale * float(q[b, i, h] @ k)
+                assert_close(lse[b, i, h], s + math.log(n), tol, "equal keys lse")
+
+
+def check_one_hot_values(lib, tol=1e-12):
+    """V rows one-hot (v_j = e_j) -> out[:, j] is the softmax probability."""
+    wl = W.Workload(name="one_hot", batch=1, num_q_heads=2, num_kv_heads=1,
+                    head_dim=32, page_size=4, kv_lens=("fixed", [23]),
+                    route="dense", seed=22)
+    inp = W.generate(wl)
+    L, D = 23, 32
+    eye = torch.zeros((1, L, D), dtype=torch.bfloat16)
+    eye[0, torch.arange(L), torch.arange(L)] = 1.0
+    pt = inp["page_table"][0]
+    vp = inp["v_pages"]
+    for j in range(L):
+        vp[int(pt[j // 4]), 0, j % 4] = eye[0, j]
+    out, _ = run_oracle(inp, lib)
+    K = inp["k_dense"][0].to(torch.float64).numpy()[0]
+    q = inp["q"].to(torch.float64).numpy()
+    for h in range(2):
+        probs = softmax(W.scale_of(wl) * (K @ q[0, 0, h]))
+        assert_close(out[0, 0, h, :L], probs, tol, "one-hot probabilities")
+        assert_close(out[0, 0, h, L:], np.zeros(D - L), tol, "one-hot tail")
+
+
+def check_poison_is_never_read(wl, lib):
+    """NaN-filled unused pages, tails and invisible keys give the same result
+    as the same slots holding zeros, and the result is finite."""
+    inp = W.generate(wl)
+    out0, lse0 = run_oracle(inp, lib)
+    clean = dict(inp)
+    for key in ("k_pages", "v_pages"):
+        x = inp[key].clone()
+        if wl.kv_dtype == W.KV_BF16:
+            x[torch.isnan(x.float())] = 0
+        else:
+            x[(x == W.E4M3_NAN_CODE) | (x == 0xFF)] = 0
+        clean[key] = x
+    out1, lse1 = run_oracle(clean, lib)
+    assert np.isfinite(out0).all(), f"{wl.name}: poisoned slots reached out"
+    assert np.array_equal(out0, out1) and np.array_equal(lse0, lse1)
+
+
+def load_golden(name):
+    with open(os.path.join(GOLDEN, name + ".json")) as f:
+        return json.load(f)
+
+
+def check_golden(name, lib):
+    g = load_golden(name)
+    u16 = np.uint16
+    q = np.array(g["q_bits"], dtype=u16)
+    kp = np.array(g["k_pages_bits"], dtype=u16)
+    vp = np.array(g["v_pages_bits"], dtype=u16)
+    scale = g["scale"]
+    if scale == "float32(ln 3)":
+        scale = float(np.float32(math.log(3.0)))
+    out, lse = orc.paged_decode_attn(
+        q, kp, vp, np.array(g["page_table"], dtype=np.int32),
+        np.array(g["kv_lens"], dtype=np.int32), num_kv_heads=g["num_kv_heads"],
+        page_size=g["page_size"], scale=scale, causal_offset=g["causal_offset"],
+        window=g["window"], kv_dtype=g["kv_dtype"], lib=lib)
+    exp_lse = np.array([[[float(x) for x in r] for r in b] for b in g["expected_lse"]])
+    assert_close(out, np.array(g["expected_out"], dtype=np.float64), g["tolerance"], name)
+    assert_close(lse, exp_lse, g["tolerance"], name)
+
+
+GOLDEN_NAMES = ["two_keys", "window_causal_equal_keys", "gqa_single_key", "empty_row"]
+
+
+def run_all(lib):
+    """Every check once; raises AssertionError at the first failure."""
+    check_decode_bf16(lib)
+    check_decode_e4m3(lib)
+    for name in GOLDEN_NAMES:
+        check_golden(name, lib)
+    for wl in SMALL_CASES:
+        check_bruteforce(wl, lib)
+    check_page_permutation(SMALL_CASES[1], lib)
+    check_split_merge(SMALL_CASES[3], [33, 70], lib)
+    check_equal_keys(lib)
+    check_one_hot_values(lib)
+    check_poison_is_never_read(SMALL_CASES[3], lib)

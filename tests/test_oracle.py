@@ -1,0 +1,152 @@
+"""The fp64 oracle against its pins (CPU only)."""
+
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import oracle as orc
+from paged_kv_decode_30_b200 import workloads as W
+from tests import oracle_pins as pins
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return orc.load()
+
+
+def test_bf16_decode_matches_torch(lib):
+    pins.check_decode_bf16(lib)
+
+
+def test_e4m3_decode_matches_torch_and_format(lib):
+    pins.check_decode_e4m3(lib)
+
+
+@pytest.mark.parametrize("name", pins.GOLDEN_NAMES)
+def test_golden(lib, name):
+    pins.check_golden(name, lib)
+
+
+@pytest.mark.parametrize("wl", pins.SMALL_CASES, ids=lambda w: w.name)
+def test_bruteforce_dense_attention(lib, wl):
+    pins.check_bruteforce(wl, lib)
+
+
+@pytest.mark.parametrize("wl", pins.SMALL_CASES[:4] + pins.SMALL_CASES[6:7], ids=lambda w: w.name)
+def test_page_permutation_is_bit_identical(lib, wl):
+    pins.check_page_permutation(wl, lib)
+
+
+@pytest.mark.parametrize("cuts", [[1], [37], [64, 65], [16, 48, 96], [0, 500]])
+def test_split_merge_equals_unsplit(lib, cuts):
+    pins.check_split_merge(pins.SMALL_CASES[3], cuts, lib)
+    pins.check_split_merge(pins.SMALL_CASES[6], cuts, lib)
+
+
+def test_equal_keys_mean_of_values(lib):
+    pins.check_equal_keys(lib)
+
+
+def test_one_hot_values_give_probabilities(lib):
+    pins.check_one_hot_values(lib)
+
+
+@pytest.mark.parametrize("wl", [pins.SMALL_CASES[0], pins.SMALL_CASES[3],
+                                pins.SMALL_CASES[5], pins.SMALL_CASES[6]],
+                         ids=lambda w: w.name)
+def test_poisoned_slots_are_never_read(lib, wl):
+    pins.check_poison_is_never_read(wl, lib)
+
+
+def test_single_key_returns_value(lib):
+    wl = W.Workload(name="single", batch=3, num_q_heads=4, num_kv_heads=2,
+                    head_dim=16, page_size=4, kv_lens=("fixed", [1, 1, 1]),
+                    route="dense", seed=31)
+    inp = W.generate(wl)
+    out, lse = pins.run_oracle(inp, lib)
+    q = inp["q"].double().numpy()
+    for b in range(3):
+        V = inp["v_dense"][b].double().numpy()
+        K = inp["k_dense"][b].double().numpy()
+        for h in range(4):
+            g = h // 2
+            np.testing.assert_array_equal(out[b, 0, h], V[g, 0])
+            s = W.scale_of(wl) * float(q[b, 0, h] @ K[g, 0])
+            assert abs(lse[b, 0, h] - s) <= 1e-12
+
+
+def test_merge_single_state_is_identity(lib):
+    rng = np.random.default_rng(0)
+    o = rng.standard_normal((1, 5, 8))
+    ls = rng.standard_normal((1, 5))
+    mo, ml = orc.merge_states(o, ls, lib=lib)
+    pins.assert_close(mo, o[0], 1e-15, "identity out")
+    pins.assert_close(ml, ls[0], 1e-15, "identity lse")
+
+
+def test_merge_ignores_empty_states(lib):
+    rng = np.random.default_rng(1)
+    o = rng.standard_normal((3, 4, 8))
+    ls = rng.standard_normal((3, 4))
+    ls[1] = -np.inf
+    o[1] = np.nan  # an empty state's output must never be read
+    mo, ml = orc.merge_states(o, ls, lib=lib)
+    ref_o, ref_l = orc.merge_states(o[[0, 2]], ls[[0, 2]], lib=lib)
+    np.testing.assert_array_equal(mo, ref_o)
+    np.testing.assert_array_equal(ml, ref_l)
+    ls[:] = -np.inf
+    mo, ml = orc.merge_states(o, ls, lib=lib)
+    assert (mo == 0).all() and np.isneginf(ml).all()
+
+
+def test_workload_recipes_match_stated_shapes():
+    """The generator's large recipes produce the stated sizes (host only)."""
+    import torch
+    gen = torch.Generator().manual_seed(W.VARLEN.seed)
+    lens = W._draw_kv_lens(W.VARLEN, gen)
+    assert lens.min() >= 512 and lens.max() <= 4096 and lens.numel() == 32
+    lens = W._draw_kv_lens(W.FP8_VERIFY, torch.Generator().manual_seed(W.FP8_VERIFY.seed))
+    assert lens.min() >= 128 and lens.max() <= 32768 and lens.numel() == 64
+    assert W.visible_token_count(W.HEADLINE, [8192] * 128) == 128 * 8192
+    # bottom-right rows with a window of 4096 see at most 4096 + 3 keys
+    assert W.visible_token_count(W.FP8_VERIFY, [10000]) == 4099
+    assert W.visible_token_count(W.FP8_VERIFY, [100]) == 100
+
+
+# --------------------------------------------------------------------------
+# Planted mistakes: each mutated copy of the oracle must fail the pins.
+
+MUTATIONS = {
+    "gqa_mapping": ("const int g = h / G;", "const int g = h % Hkv;"),
+    "window_off_by_one": ("pos - (int64_t)window + 1", "pos - (int64_t)window"),
+    "causal_strict": ("if (causal && j > pos) return 0;", "if (causal && j >= pos) return 0;"),
+    "lse_drops_max": ("const double row_lse = m + log(sum);", "const double row_lse = log(sum);"),
+    "page_row_swapped": ("const int64_t row = j % page_size;", "const int64_t row = j / page_size;"),
+    "scale_dropped": ("s[j] = dscale * dot;", "s[j] = dot;"),
+    "e4m3_bias": ("mag = ldexp(1.0 + (double)m / 8.0, e - 7);",
+                  "mag = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "merge_weight": ("const double w = exp(ls - total);", "const double w = exp(ls - m);"),
+    "bottom_right_shift": ("return kv_len - (int64_t)q_len + i;", "return kv_len - (int64_t)q_len + i - 1;"),
+    "kv_scale_dropped": ("* kv_scale;\n}", ";\n}"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(tmp_path, name):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = open(orc._SRC).read()
+    old, new = MUTATIONS[name]
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new)
+    c = tmp_path / "oracle_mut.c"
+    c.write_text(mutated)
+    so = tmp_path / "liboracle_mut.so"
+    subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared",
+                    str(c), "-o", str(so), "-lm"], check=True)
+    mlib = orc.load(str(so))
+    with pytest.raises(AssertionError):
+        pins.run_all(mlib)
