@@ -1,0 +1,186 @@
+/*
+ * paged_decode_attn: paged-KV decode attention for NVIDIA B200 (sm_100a).
+ *
+ * The operation (one decode step of one attention layer): for every sequence
+ * b, query row i and query head h, softmax attention of q[b, i, h, :] over the
+ * keys of sequence b, with K/V rows gathered through a page table:
+ *
+ *   s_j   = scale * q . k_j              for every key j the row may see
+ *   lse   = ln sum_j exp(s_j)
+ *   out   = sum_j exp(s_j - lse) * v_j
+ *
+ * Sources (page title, section):
+ *  - "AstrAI commit log, attn_paged_decode_split_kv_mma.cuh": split-KV paged
+ *    decode; per-position page-table lookup when loading K/V tiles; GQA head
+ *    packing; causal_offset (-1 off, >= 0 first query position); split
+ *    partials written without a memset; compute_num_splits.
+ *  - "b12x 0.30.0, Kernel inventory, Attention table, Paged attention row":
+ *    bf16 and FP8-E4M3 KV caches, split-KV or direct output, sliding window,
+ *    GQA, and a persistent merge kernel for the split partials.
+ *  - "sglang profiler skill, fuse-overlap catalog, vLLM-origin attention +
+ *    output quant row": merge_attn_states merges attention states by LSE.
+ *
+ * Where the pages leave the operation open, this library takes:
+ *  - lse is a natural logarithm.
+ *  - causal_offset = PDA_CAUSAL_BOTTOM_RIGHT (-2) aligns query row i of
+ *    sequence b at position kv_lens[b] - q_len + i (speculative verify rows).
+ *  - a window of W keys includes the query's own position: key j is visible
+ *    to a row at position pos iff j >= pos - W + 1; window <= 0 is off; with
+ *    causal off the window is measured from kv_lens[b] - 1.
+ *  - query head h reads kv head h / (num_q_heads / num_kv_heads).
+ *  - KV pools are laid out [num_pages, num_kv_heads, page_size, head_dim].
+ *  - FP8: element value = e4m3 code * kv_scale, one scale shared by K and V.
+ *  - a row that sees no key gets out = 0 and lse = -inf.
+ *
+ * All entry points return a status and never abort or throw. Device work is
+ * asynchronous on the given stream; no entry point synchronises except
+ * pda_last_device_error.
+ */
+#ifndef PAGED_DECODE_ATTN_H_
+#define PAGED_DECODE_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PDA_API __attribute__((visibility("default")))
+#else
+#define PDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st* pda_stream_t;
+
+#define PDA_ABI_VERSION 1
+
+typedef enum {
+  PDA_KV_BF16 = 0,      /* K/V elements are bfloat16 */
+  PDA_KV_FP8_E4M3 = 1   /* K/V elements are FP8 E4M3 codes (uint8) */
+} pda_kv_dtype;
+
+typedef enum {
+  PDA_OK = 0,
+  PDA_ERR_INVALID_ARG = 1,  /* a size, pointer or field is out of range */
+  PDA_ERR_UNSUPPORTED = 2,  /* valid, but no kernel variant for it */
+  PDA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+  PDA_ERR_WORKSPACE = 4,    /* caller workspace too small / allocation failed */
+  PDA_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+  PDA_ERR_BAD_PAGE = 6,     /* device saw a page id or kv_len out of range */
+  PDA_ERR_TIMEOUT = 7       /* device gave up waiting on a copy */
+} pda_status;
+
+#define PDA_CAUSAL_OFF (-1)           /* no causal mask */
+#define PDA_CAUSAL_BOTTOM_RIGHT (-2)  /* row i at kv_lens[b] - q_len + i */
+
+/* flags */
+#define PDA_FLAG_NO_PDL 1u  /* launch the merge without programmatic dependent launch */
+
+typedef struct {
+  int32_t batch;            /* B >= 0 */
+  int32_t q_len;            /* query rows per sequence, 1..8 */
+  int32_t num_q_heads;      /* Hq, a multiple of num_kv_heads */
+  int32_t num_kv_heads;     /* Hkv >= 1 */
+  int32_t head_dim;         /* D in {64, 128, 256} */
+  int32_t page_size;        /* P, a power of two in [8, 256] */
+  int32_t max_pages_per_seq;/* row stride of page_table; kv_lens[b] <= this * P */
+  int32_t num_pages;        /* pages in each pool; page ids must be < this */
+  float scale;              /* softmax scale (> 0), e.g. 1/sqrt(D) */
+  int32_t causal_offset;    /* PDA_CAUSAL_OFF, PDA_CAUSAL_BOTTOM_RIGHT, or >= 0 */
+  int32_t window;           /* <= 0 off; else keys j >= pos - window + 1 */
+  int32_t kv_dtype;         /* pda_kv_dtype */
+  float kv_scale;           /* FP8 only: value = code * kv_scale (> 0) */
+  int32_t max_kv_len;       /* host hint, >= every kv_lens[b]; 0 -> max_pages_per_seq * P.
+                               Used only to choose the split count. */
+  int32_t num_splits;       /* 0 -> heuristic; > 0 forces this many KV splits */
+  uint32_t flags;           /* PDA_FLAG_* */
+  void* workspace;          /* device scratch for split partials, or NULL */
+  size_t workspace_bytes;   /* size of workspace */
+  int32_t* num_splits_out;  /* optional host out: split count used */
+} pda_params;
+
+/*
+ * Paged decode attention.
+ *
+ * q           device, bf16 [B, q_len, Hq, D], contiguous.
+ * k_pages     device, [num_pages, Hkv, P, D] of bf16 (PDA_KV_BF16) or uint8
+ * v_pages     e4m3 codes (PDA_KV_FP8_E4M3), contiguous.
+ * page_table  device, int32 [B, max_pages_per_seq]; entry t of row b is the
+ *             pool page holding keys [t*P, (t+1)*P) of sequence b. Entries
+ *             past ceil(kv_lens[b] / P) are never read (may hold -1).
+ * kv_lens     device, int32 [B], keys per sequence (0 allowed).
+ * params      host, read during the call only.
+ * out         device, fp32 [B, q_len, Hq, D].
+ * lse         device, fp32 [B, q_len, Hq], natural log; may be NULL.
+ * stream      CUDA stream for all device work.
+ *
+ * Inputs are read only. Slots of a page past kv_lens[b], and keys no row
+ * may see, are never weighted (their bytes may be NaN). q, k_pages, v_pages
+ * and out must be 16-byte aligned; page_table, kv_lens and lse 4-byte
+ * aligned; a caller workspace 256-byte aligned (else PDA_ERR_MISALIGNED).
+ *
+ * Workspace: when the call splits the KV range (num_splits > 1) it needs
+ * paged_decode_attn_workspace_bytes(params) bytes of device scratch. If
+ * params->workspace is NULL the library uses a grow-only buffer it owns, one
+ * per device, shared by every call on that device: calls that may overlap on
+ * different streams must pass their own workspace. The library never
+ * clears the workspace; every slot the kernels read was written earlier in
+ * the same call.
+ *
+ * Errors: invalid sizes or pointers return before any device work. A page
+ * id >= num_pages or < 0 met on the device is never dereferenced; the kernel
+ * records PDA_ERR_BAD_PAGE in a device error word (see pda_last_device_error)
+ * and the affected output is unspecified.
+ */
+PDA_API pda_status paged_decode_attn(const void* q, const void* k_pages,
+                             const void* v_pages, const int32_t* page_table,
+                             const int32_t* kv_lens, const pda_params* params,
+                             float* out, float* lse, pda_stream_t stream);
+
+/* Bytes of workspace paged_decode_attn needs for these params with the
+ * split count it would choose (0 when it would not split). SIZE_MAX if the
+ * params are invalid. */
+PDA_API size_t paged_decode_attn_workspace_bytes(const pda_params* params);
+
+/* The split count paged_decode_attn would use for these params on a device
+ * with num_sms SMs (host-only; the heuristic of the split planner). Returns
+ * a value >= 1, or 0 if params are invalid. */
+PDA_API int32_t pda_choose_num_splits(const pda_params* params, int32_t num_sms);
+
+/*
+ * LSE merge of split partials, the merge step on its own (merge_attn_states /
+ * PagedPersistentMergeKernel):
+ *   lse[r]    = m + ln sum_s exp(lse_parts[s, r] - m),  m = max_s lse_parts[s, r]
+ *   out[r, :] = sum_s exp(lse_parts[s, r] - lse[r]) * o_parts[s, r, :]
+ * A row whose every part has lse = -inf gets out = 0 and lse = -inf, and
+ * o_parts of such parts are not read.
+ *
+ * o_parts    device fp32 [num_splits, rows, head_dim]
+ * lse_parts  device fp32 [num_splits, rows]
+ * out        device fp32 [rows, head_dim];  lse device fp32 [rows] or NULL
+ * head_dim in {64, 128, 256}; num_splits >= 1; o_parts and out 16-byte
+ * aligned, lse_parts and lse 4-byte aligned.
+ */
+PDA_API pda_status pda_merge_states(const float* o_parts, const float* lse_parts,
+                            int32_t num_splits, int64_t rows, int32_t head_dim,
+                            float* out, float* lse, pda_stream_t stream);
+
+/* Human-readable name of a status. Never NULL. */
+PDA_API const char* pda_status_string(pda_status status);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word: PDA_ERR_BAD_PAGE or PDA_ERR_TIMEOUT if a kernel recorded one since
+ * the last read, PDA_OK otherwise (PDA_ERR_CUDA if the sync failed). */
+PDA_API pda_status pda_last_device_error(pda_stream_t stream);
+
+/* PDA_ABI_VERSION of the loaded library. */
+PDA_API int32_t pda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_DECODE_ATTN_H_ */

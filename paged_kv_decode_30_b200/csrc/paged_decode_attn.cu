@@ -1,0 +1,340 @@
+// Host side of the paged decode attention library: argument validation, the
+// split planner, workspace, kernel dispatch and the exported C ABI.
+//
+// Sources: "AstrAI commit log, attn_paged_decode_split_kv_mma.cuh"
+// (compute_num_splits / alloc_split_partials / dispatch_head_dim host
+// helpers; the split kernel writes every partial slot it owns, so partials
+// are never cleared) and "b12x 0.30.0, Kernel inventory, Attention table,
+// Paged attention row" (split-KV or direct output; separate merge kernel).
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "merge.cuh"
+#include "paged_decode_attn.h"
+#include "split_variants.cuh"
+
+namespace pda {
+
+// One device error word per device that loads the library.
+__device__ int g_error_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+// Modelled cost of the merge launch, in units of one CTA iteration
+// (NW warp tiles, ~64 KB of K/V at the per-SM share of HBM bandwidth).
+constexpr int kMergeCostIters = 2;
+// Fixed cost of one CTA (pipeline fill: the first tiles' copy latency, the
+// page-id prefetch, the epilogue), in the same units.
+constexpr int kCtaFillIters = 1;
+constexpr int kMaxSplits = 128;
+
+struct DeviceState {
+  bool init = false;
+  int num_sms = 0;
+  int* err = nullptr;        // device address of g_error_word
+  void* ws = nullptr;        // library-owned workspace (grow-only)
+  size_t ws_bytes = 0;
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+pda_status device_state(DeviceState** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return PDA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.init) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return PDA_ERR_CUDA;
+    void* err = nullptr;
+    if (cudaGetSymbolAddress(&err, g_error_word) != cudaSuccess) return PDA_ERR_CUDA;
+    st.num_sms = sms;
+    st.err = static_cast<int*>(err);
+    st.init = true;
+  }
+  *out = &st;
+  return PDA_OK;
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int ilog2(int x) { int l = 0; while ((1 << l) < x) ++l; return l; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// Static shape of the launch that a params struct leads to.
+struct Plan {
+  int G, M, mt, row_tiles, tw, elt;
+  long long rows;          // B * q_len * Hq
+  int tiles_per_cta_iter;  // tokens one CTA iteration covers = tw * warps
+};
+
+pda_status validate(const pda_params* p) {
+  if (p == nullptr) return PDA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->q_len < 1 || p->num_q_heads < 1 || p->num_kv_heads < 1)
+    return PDA_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return PDA_ERR_INVALID_ARG;
+  if (p->head_dim < 1 || p->page_size < 1 || p->max_pages_per_seq < 1 || p->num_pages < 1)
+    return PDA_ERR_INVALID_ARG;
+  if (!(p->scale > 0.f) || !std::isfinite(p->scale)) return PDA_ERR_INVALID_ARG;
+  if (p->causal_offset < PDA_CAUSAL_BOTTOM_RIGHT) return PDA_ERR_INVALID_ARG;
+  if (p->kv_dtype != PDA_KV_BF16 && p->kv_dtype != PDA_KV_FP8_E4M3) return PDA_ERR_INVALID_ARG;
+  if (p->kv_dtype == PDA_KV_FP8_E4M3 && (!(p->kv_scale > 0.f) || !std::isfinite(p->kv_scale)))
+    return PDA_ERR_INVALID_ARG;
+  if (p->max_kv_len < 0 || p->num_splits < 0) return PDA_ERR_INVALID_ARG;
+  if ((long long)p->max_pages_per_seq * p->page_size > INT_MAX) return PDA_ERR_INVALID_ARG;
+  // supported variants
+  if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256) return PDA_ERR_UNSUPPORTED;
+  if (!is_pow2(p->page_size) || p->page_size < 8 || p->page_size > 256) return PDA_ERR_UNSUPPORTED;
+  if (p->q_len > 8) return PDA_ERR_UNSUPPORTED;
+  if (p->batch > 65535) return PDA_ERR_UNSUPPORTED;
+  return PDA_OK;
+}
+
+Plan make_plan(const pda_params* p) {
+  Plan pl{};
+  pl.G = p->num_q_heads / p->num_kv_heads;
+  pl.M = pl.G * p->q_len;
+  pl.mt = pl.M >= 8 ? 8 : (pl.M >= 4 ? 4 : (pl.M >= 2 ? 2 : 1));
+  pl.row_tiles = (int)cdiv(pl.M, pl.mt);
+  const int tw_full = 8 * (32 / (p->head_dim / 8));
+  pl.tw = p->page_size < tw_full ? p->page_size : tw_full;
+  pl.elt = p->kv_dtype == PDA_KV_BF16 ? 2 : 1;
+  pl.rows = (long long)p->batch * p->q_len * p->num_q_heads;
+  pl.tiles_per_cta_iter = pl.tw * kFmaWarps;
+  return pl;
+}
+
+int choose_splits(const pda_params* p, const Plan& pl, int num_sms) {
+  const long long len_bound =
+      p->max_kv_len > 0 ? p->max_kv_len : (long long)p->max_pages_per_seq * p->page_size;
+  // Keys one row tile can see: bounded by the window (plus the spread of the
+  // tile's query positions) when a window is set.
+  long long span = len_bound;
+  if (p->window > 0) span = std::min<long long>(span, (long long)p->window + p->q_len);
+  const long long max_tiles = std::max<long long>(1, cdiv(span, pl.tw));
+  if (p->num_splits > 0) return (int)std::min<long long>(p->num_splits, std::min<long long>(max_tiles, kMaxSplits));
+  const long long iters = std::max<long long>(1, cdiv(span, pl.tiles_per_cta_iter));
+  const long long units = (long long)p->batch * p->num_kv_heads * pl.row_tiles;
+  const long long slots = std::max(1, num_sms);  // one CTA per SM
+  long long best_cost = LLONG_MAX;
+  int best = 1;
+  const long long smax = std::min<long long>(std::min<long long>(iters, max_tiles), kMaxSplits);
+  for (long long s = 1; s <= smax; ++s) {
+    if (s * p->num_kv_heads > 65535) break;
+    const long long waves = cdiv(units * s, slots);
+    const long long cost =
+        waves * (cdiv(iters, s) + kCtaFillIters) + (s > 1 ? kMergeCostIters : 0);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = (int)s;
+    }
+  }
+  return best;
+}
+
+size_t partial_bytes(const Plan& pl, int splits, int D, size_t* lse_offset) {
+  const size_t o_bytes = (size_t)splits * (size_t)pl.rows * (size_t)D * sizeof(float);
+  const size_t off = (o_bytes + 255) / 256 * 256;
+  if (lse_offset) *lse_offset = off;
+  return off + (size_t)splits * (size_t)pl.rows * sizeof(float);
+}
+
+}  // namespace
+
+cudaError_t launch_merge(int D, const float* o_parts, const float* lse_parts,
+                         int num_splits, long long rows, float* out, float* lse,
+                         cudaStream_t stream, bool pdl) {
+  if (rows <= 0) return cudaSuccess;
+  constexpr int kWarpsPerBlock = 8;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)cdiv(rows, kWarpsPerBlock));
+  cfg.blockDim = dim3(kWarpsPerBlock * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  switch (D) {
+    case 64: return cudaLaunchKernelEx(&cfg, merge_states_kernel<64>, o_parts, lse_parts, num_splits, rows, out, lse);
+    case 128: return cudaLaunchKernelEx(&cfg, merge_states_kernel<128>, o_parts, lse_parts, num_splits, rows, out, lse);
+    case 256: return cudaLaunchKernelEx(&cfg, merge_states_kernel<256>, o_parts, lse_parts, num_splits, rows, out, lse);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace pda
+
+using namespace pda;
+
+extern "C" {
+
+int32_t pda_abi_version(void) { return PDA_ABI_VERSION; }
+
+const char* pda_status_string(pda_status s) {
+  switch (s) {
+    case PDA_OK: return "ok";
+    case PDA_ERR_INVALID_ARG: return "invalid argument";
+    case PDA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PDA_ERR_MISALIGNED: return "misaligned pointer";
+    case PDA_ERR_WORKSPACE: return "workspace too small or allocation failed";
+    case PDA_ERR_CUDA: return "CUDA error";
+    case PDA_ERR_BAD_PAGE: return "page id or kv length out of range (device)";
+    case PDA_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int32_t pda_choose_num_splits(const pda_params* params, int32_t num_sms) {
+  if (validate(params) != PDA_OK || num_sms < 1) return 0;
+  return choose_splits(params, make_plan(params), num_sms);
+}
+
+size_t paged_decode_attn_workspace_bytes(const pda_params* params) {
+  if (validate(params) != PDA_OK) return SIZE_MAX;
+  const Plan pl = make_plan(params);
+  int sms = 148;
+  DeviceState* st = nullptr;
+  if (params->num_splits == 0 && device_state(&st) == PDA_OK) sms = st->num_sms;
+  const int s = choose_splits(params, pl, sms);
+  return s > 1 ? partial_bytes(pl, s, params->head_dim, nullptr) : 0;
+}
+
+pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_pages,
+                             const int32_t* page_table, const int32_t* kv_lens,
+                             const pda_params* params, float* out, float* lse,
+                             pda_stream_t stream_) {
+  pda_status st = validate(params);
+  if (st != PDA_OK) return st;
+  const pda_params& p = *params;
+  if (p.batch == 0) {
+    if (p.num_splits_out) *p.num_splits_out = 1;
+    return PDA_OK;
+  }
+  if (!q || !k_pages || !v_pages || !page_table || !kv_lens || !out) return PDA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+      !aligned(page_table, 4) || !aligned(kv_lens, 4) || (lse && !aligned(lse, 4)))
+    return PDA_ERR_MISALIGNED;
+  if (p.workspace && !aligned(p.workspace, 256)) return PDA_ERR_MISALIGNED;
+
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != PDA_OK) return st;
+
+  const Plan pl = make_plan(params);
+  const int splits = choose_splits(params, pl, dev->num_sms);
+  if ((long long)splits * p.num_kv_heads > 65535) return PDA_ERR_UNSUPPORTED;
+
+  SplitArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.k_pages = static_cast<const uint8_t*>(k_pages);
+  a.v_pages = static_cast<const uint8_t*>(v_pages);
+  a.page_table = page_table;
+  a.kv_lens = kv_lens;
+  a.out = out;
+  a.lse = lse;
+  a.err = dev->err;
+  a.B = p.batch;
+  a.Lq = p.q_len;
+  a.Hq = p.num_q_heads;
+  a.Hkv = p.num_kv_heads;
+  a.G = pl.G;
+  a.M = pl.M;
+  a.page_size = p.page_size;
+  a.log2_page = ilog2(p.page_size);
+  a.max_pages = p.max_pages_per_seq;
+  a.num_pages = p.num_pages;
+  a.tile_shift = ilog2(p.page_size / pl.tw);
+  a.num_splits = splits;
+  a.row_tiles = pl.row_tiles;
+  a.causal_offset = p.causal_offset;
+  a.window = p.window;
+  const float log2e = 1.4426950408889634f;
+  const bool fp8 = p.kv_dtype == PDA_KV_FP8_E4M3;
+  a.qk_scale_log2 = p.scale * log2e * (fp8 ? p.kv_scale : 1.f);
+  a.v_scale = fp8 ? p.kv_scale : 1.f;
+  a.head_stride = (long long)p.page_size * p.head_dim * pl.elt;
+  a.page_stride = a.head_stride * p.num_kv_heads;
+
+  if (splits > 1) {
+    size_t lse_off = 0;
+    const size_t need = partial_bytes(pl, splits, p.head_dim, &lse_off);
+    void* ws = p.workspace;
+    if (ws == nullptr) {
+      std::lock_guard<std::mutex> lock(g_mu);
+      if (dev->ws_bytes < need) {
+        if (dev->ws) cudaFree(dev->ws);  // synchronises the device
+        dev->ws = nullptr;
+        dev->ws_bytes = 0;
+        if (cudaMalloc(&dev->ws, need) != cudaSuccess) {
+          dev->ws = nullptr;
+          return PDA_ERR_WORKSPACE;
+        }
+        dev->ws_bytes = need;
+      }
+      ws = dev->ws;
+    } else if (p.workspace_bytes < need) {
+      return PDA_ERR_WORKSPACE;
+    }
+    a.o_part = static_cast<float*>(ws);
+    a.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + lse_off);
+  }
+
+  const dim3 grid((unsigned)pl.row_tiles, (unsigned)(splits * p.num_kv_heads), (unsigned)p.batch);
+  cudaError_t e;
+  const int kv = fp8 ? 1 : 0;
+  switch (p.head_dim) {
+    case 64: e = launch_split_d64(kv, pl.mt, pl.tw, a, grid, stream); break;
+    case 128: e = launch_split_d128(kv, pl.mt, pl.tw, a, grid, stream); break;
+    case 256: e = launch_split_d256(kv, pl.mt, pl.tw, a, grid, stream); break;
+    default: e = cudaErrorNotSupported;
+  }
+  if (e == cudaErrorNotSupported) return PDA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return PDA_ERR_CUDA;
+  if (splits > 1) {
+    e = launch_merge(p.head_dim, a.o_part, a.lse_part, splits, pl.rows, out, lse, stream,
+                     (p.flags & PDA_FLAG_NO_PDL) == 0);
+    if (e != cudaSuccess) return PDA_ERR_CUDA;
+  }
+  if (p.num_splits_out) *p.num_splits_out = splits;
+  return PDA_OK;
+}
+
+pda_status pda_merge_states(const float* o_parts, const float* lse_parts, int32_t num_splits,
+                            int64_t rows, int32_t head_dim, float* out, float* lse,
+                            pda_stream_t stream) {
+  if (num_splits < 1 || rows < 0) return PDA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PDA_ERR_UNSUPPORTED;
+  if (rows == 0) return PDA_OK;
+  if (!o_parts || !lse_parts || !out) return PDA_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) || (lse && !aligned(lse, 4)))
+    return PDA_ERR_MISALIGNED;
+  const cudaError_t e = launch_merge(head_dim, o_parts, lse_parts, num_splits, rows, out, lse,
+                                     reinterpret_cast<cudaStream_t>(stream), false);
+  return e == cudaSuccess ? PDA_OK : PDA_ERR_CUDA;
+}
+
+pda_status pda_last_device_error(pda_stream_t stream) {
+  DeviceState* dev = nullptr;
+  pda_status st = device_state(&dev);
+  if (st != PDA_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PDA_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return PDA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return PDA_ERR_CUDA;
+  return static_cast<pda_status>(word);
+}
+
+}  // extern "C"

@@ -1,0 +1,510 @@
+// Split-KV paged decode kernel, CUDA-core (FMA) path for small packed-row
+// counts (M = G * q_len rows per kv head, M_T <= 8 rows per CTA).
+//
+// Sources: "AstrAI commit log, attn_paged_decode_split_kv_mma.cuh" (scalar
+// variant: page table resolved per position while loading the K/V tile;
+// multi-stage copy pipeline keeping STAGES-1 tiles in flight; predicated
+// partial tiles; split partials written without a memset), "b12x 0.30.0,
+// Kernel inventory, Attention table, Paged attention row" (bf16 and
+// FP8-E4M3 KV, sliding window, GQA, split-KV or direct output).
+//
+// B200 design:
+//  * One CTA per (row tile, split, kv head, sequence). The CTA's key range is
+//    dealt to its NW warps tile by tile (warp w takes tiles w, w+NW, ...).
+//    Each warp owns a STAGES-deep ring of K/V tiles in shared memory, filled
+//    by untiled bulk copies (one per K tile, one per V tile: a tile is TW
+//    consecutive tokens of one page, a contiguous block of the HND pool)
+//    that complete on the warp's own mbarriers. No CTA-wide barrier sits in
+//    the main loop.
+//  * Page ids for the warp's next 64 tiles live in registers (one per lane,
+//    two batches), so the lookup latency never sits in front of a copy.
+//    A page id outside [0, num_pages) is recorded as an error and replaced by
+//    page 0, so no access ever leaves the pool.
+//  * Lane layout: a token's D elements are split over LPT = D/8 lanes, 8
+//    elements (one 16-byte bf16 or 8-byte e4m3 load) per lane; TPI = 32/LPT
+//    tokens are read per warp instruction (a warp reads 512 contiguous bytes
+//    for bf16, conflict-free). Q sits in registers, pre-scaled by
+//    scale*log2(e) (and kv_scale for FP8), for the lane's 8 elements of each
+//    of the M_T rows.
+//  * Scores: 8*M_T partial dot products per lane per group of 8 tokens are
+//    summed over the LPT lanes of a token with a reduce-scatter butterfly
+//    (each step halves the values a lane carries), so a score costs about one
+//    shuffle instead of log2(LPT).
+//  * Online softmax in fp32 with exp2; probabilities go through a small
+//    per-warp shared buffer to the P.V loop, which keeps acc[M_T][8] fp32 per
+//    lane.
+//  * Masking by select, never by multiplying: scores of invisible keys become
+//    -inf; V of keys no row can see is zeroed before the FMA, so NaN bytes in
+//    tail slots or outside the window never reach the output. Tiles fully
+//    inside every row's visible range skip all mask work.
+//  * End: the warps' (m, l, acc) are merged through shared memory; the CTA
+//    writes out/lse directly (one split) or normalised partials (several).
+#pragma once
+
+#include "pda_device.cuh"
+
+namespace pda {
+
+struct SplitArgs {
+  const uint16_t* q;         // bf16 bits [B, Lq, Hq, D]
+  const uint8_t* k_pages;    // pool bytes [num_pages, Hkv, P, D]
+  const uint8_t* v_pages;
+  const int32_t* page_table; // [B, max_pages]
+  const int32_t* kv_lens;    // [B]
+  float* out;                // [B, Lq, Hq, D]       (num_splits == 1)
+  float* lse;                // [B, Lq, Hq] or null  (num_splits == 1)
+  float* o_part;             // [S, B, Lq, Hq, D]    (num_splits > 1)
+  float* lse_part;           // [S, B, Lq, Hq]
+  int* err;                  // device error word
+  int B, Lq, Hq, Hkv, G, M;
+  int page_size, log2_page, max_pages, num_pages;
+  int tile_shift;            // log2(page_size / TW): tiles per page
+  int num_splits, row_tiles;
+  int causal_offset, window;
+  float qk_scale_log2;       // scale * log2(e) [* kv_scale for FP8]
+  float v_scale;             // 1, or kv_scale for FP8
+  long long page_stride;     // bytes per page: Hkv * P * D * elt
+  long long head_stride;     // bytes per (page, head) block: P * D * elt
+};
+
+template <int D, int KV, int MT, int TW, int NW, int STAGES>
+struct FmaCfg {
+  static constexpr int ELT = KV == 0 ? 2 : 1;
+  static constexpr int CH = 8;             // elements per lane chunk
+  static constexpr int LPT = D / CH;       // lanes per token
+  static constexpr int TPI = 32 / LPT;     // tokens per warp instruction
+  static constexpr int NTOK = TW / TPI;    // tokens per lane group per tile
+  static constexpr int NV = NTOK * MT;     // partial scores per lane
+  static constexpr int NVF = NV >= LPT ? NV / LPT : 1;  // after reduce-scatter
+  // distinct rows among a lane's NVF slots, and the lowest xor distance
+  // between lanes that hold the same rows (for row-wise max / sum)
+  static constexpr int NFOLD = NVF > MT ? MT : NVF;
+  static constexpr int RED_LO =
+      NV >= LPT ? (NVF >= MT ? 1 : MT / NVF) : (LPT / NV) * MT;
+  static constexpr int TILE_BYTES = TW * D * ELT;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int PBUF_FLOATS = TW * MT;
+  static constexpr int WARP_SMEM_RAW =
+      STAGES * STAGE_BYTES + 32 /*mbarriers*/ + PBUF_FLOATS * 4 + 32 /*alpha*/;
+  static constexpr int WARP_SMEM = (WARP_SMEM_RAW + 127) / 128 * 128;
+  static constexpr int MERGE_SMEM = (2 * NW * MT + NW * MT * D) * 4;
+  static constexpr int SMEM =
+      NW * WARP_SMEM > MERGE_SMEM ? NW * WARP_SMEM : MERGE_SMEM;
+  static_assert(D % 64 == 0 && D <= 256, "head_dim");
+  static_assert(TW % TPI == 0 && NTOK >= 1, "tile");
+  static_assert(STAGES <= 4, "mbarrier area holds 4");
+  static_assert(TILE_BYTES % 16 == 0, "bulk copy size");
+};
+
+// Visible key range [lo, hi) of a query row at index i (reading of the
+// causal_offset / window conventions in the public header).
+__device__ __forceinline__ void row_range(const SplitArgs& a, int L, int i,
+                                          int& lo, int& hi) {
+  long long pos;
+  if (a.causal_offset >= 0)
+    pos = (long long)a.causal_offset + i;
+  else if (a.causal_offset == -2)
+    pos = (long long)L - a.Lq + i;
+  else
+    pos = (long long)L - 1;
+  long long h = a.causal_offset != -1 ? pos + 1 : (long long)L;
+  h = h < 0 ? 0 : (h > L ? L : h);
+  long long l = a.window > 0 ? pos - a.window + 1 : 0;
+  l = l < 0 ? 0 : (l > L ? L : l);
+  lo = (int)l;
+  hi = (int)h;
+}
+
+// Butterfly reduce-scatter of N values over the lanes whose ids differ in the
+// bits of O, O/2, ..., 1: at each step a lane keeps the half of its values
+// picked by its lane bit and adds the partner's copy of that half. After
+// log2(N) steps each lane holds one value summed over 2^(steps) lanes; the
+// remaining steps are plain butterflies. Values end in v[0 .. N/lanes).
+template <int N, int O>
+__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (N > 1) {
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        const float send = up ? v[i] : v[i + N / 2];
+        const float keep = up ? v[i + N / 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, O);
+      }
+      reduce_scatter<N / 2, O / 2>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], O);
+      reduce_scatter<1, O / 2>(v, lane);
+    }
+  }
+}
+
+template <int KV>
+__device__ __forceinline__ void load_chunk(const uint8_t* p, float (&f)[8]) {
+  if constexpr (KV == 0) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    bf16x8_to_f32(u, f);
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    e4m3x8_to_f32(u, f);
+  }
+}
+
+template <int D, int KV, int MT, int TW, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32, 1)
+    split_fma_kernel(const SplitArgs a) {
+  using C = FmaCfg<D, KV, MT, TW, NW, STAGES>;
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int rt = blockIdx.x;
+  const int split = blockIdx.y % a.num_splits;
+  const int kvh = blockIdx.y / a.num_splits;
+  const int b = blockIdx.z;
+
+  uint8_t* wbase = smem + warp * C::WARP_SMEM;
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(wbase + STAGES * C::STAGE_BYTES);
+  float* pbuf = reinterpret_cast<float*>(wbase + STAGES * C::STAGE_BYTES + 32);
+  float* abuf = pbuf + C::PBUF_FLOATS;
+
+  // ---- key range of this CTA -------------------------------------------
+  int L = __ldg(a.kv_lens + b);
+  const int Lmax = a.max_pages << a.log2_page;
+  if (L < 0 || L > Lmax) {
+    if (threadIdx.x == 0) record_error_at(a.err, kErrBadPage);
+    L = L < 0 ? 0 : Lmax;
+  }
+  const int R0 = rt * MT;
+  const int Rlast = min(a.M, R0 + MT) - 1;
+  int lo_u, hi_u, lo_x, hi_x;
+  row_range(a, L, R0 / a.G, lo_u, hi_x);     // first row: union lo, intersection hi
+  row_range(a, L, Rlast / a.G, lo_x, hi_u);  // last row: intersection lo, union hi
+  const int k_begin = lo_u / TW;
+  const int k_end = hi_u > lo_u ? (hi_u + TW - 1) / TW : k_begin;
+  const int n_all = k_end - k_begin;
+  const int chunk = (n_all + a.num_splits - 1) / a.num_splits;
+  const int c0 = min(n_all, split * chunk);
+  const int c1 = min(n_all, c0 + chunk);
+  const int cta_tiles = c1 - c0;
+  const int my_tiles = cta_tiles > warp ? (cta_tiles - warp + NW - 1) / NW : 0;
+  const int kbase = k_begin + c0 + warp;  // absolute tile index of my tile 0
+
+  const int tile_shift = a.tile_shift;
+  const int tile_mask = (1 << tile_shift) - 1;
+  const int32_t* pt_row = a.page_table + (long long)b * a.max_pages;
+  const uint8_t* kbase_ptr = a.k_pages + (long long)kvh * a.head_stride;
+  const uint8_t* vbase_ptr = a.v_pages + (long long)kvh * a.head_stride;
+
+  // ---- barriers and page-id prefetch -------------------------------------
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) mbar_init(&mbar[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  auto load_pid = [&](int n) -> int {
+    if (n >= my_tiles) return 0;
+    int pid = __ldg(pt_row + ((kbase + n * NW) >> tile_shift));
+    if ((unsigned)pid >= (unsigned)a.num_pages) {
+      record_error_at(a.err, kErrBadPage);
+      pid = 0;
+    }
+    return pid;
+  };
+  int pid_cur = load_pid(lane);
+  int pid_nxt = load_pid(32 + lane);
+  int pid_batch = 0;
+
+  auto issue = [&](int n) {  // warp-uniform
+    const int nb = n >> 5;
+    if (nb != pid_batch) {
+      pid_cur = pid_nxt;
+      pid_nxt = load_pid((nb + 1) * 32 + lane);
+      pid_batch = nb;
+    }
+    const int pid = __shfl_sync(FULL, pid_cur, n & 31);
+    if (lane == 0) {
+      const int s = n % STAGES;
+      const long long off = (long long)pid * a.page_stride +
+                            (long long)((kbase + n * NW) & tile_mask) * C::TILE_BYTES;
+      uint8_t* dst = wbase + s * C::STAGE_BYTES;
+      mbar_arrive_expect_tx(&mbar[s], C::STAGE_BYTES);
+      bulk_g2s(dst, kbase_ptr + off, C::TILE_BYTES, &mbar[s]);
+      bulk_g2s(dst + C::TILE_BYTES, vbase_ptr + off, C::TILE_BYTES, &mbar[s]);
+    }
+  };
+
+  const int n_pro = my_tiles < STAGES ? my_tiles : STAGES;
+  for (int n = 0; n < n_pro; ++n) issue(n);
+
+  // ---- Q fragment ----------------------------------------------------------
+  const int grp = lane / C::LPT;
+  const int d0 = (lane % C::LPT) * C::CH;
+  float qf[MT][8];
+#pragma unroll
+  for (int r = 0; r < MT; ++r) {
+    const int R = R0 + r;
+    if (R < a.M) {
+      const int i = R / a.G, h = kvh * a.G + R % a.G;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+          a.q + ((long long)(b * a.Lq + i) * a.Hq + h) * D + d0));
+      bf16x8_to_f32(u, qf[r]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[r][e] *= a.qk_scale_log2;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[r][e] = 0.f;
+    }
+  }
+
+  // ---- slots this lane holds after the reduce-scatter --------------------
+  const int c = lane % C::LPT;
+  const int vbase = C::NV >= C::LPT ? c * C::NVF : c / (C::LPT / C::NV);
+  int slot_tok[C::NVF], slot_row[C::NVF], slot_lo[C::NVF], slot_hi[C::NVF];
+#pragma unroll
+  for (int i = 0; i < C::NVF; ++i) {
+    const int v = vbase + i;
+    slot_tok[i] = (v / MT) * C::TPI + grp;
+    slot_row[i] = v % MT;
+    const int R = R0 + slot_row[i];
+    if (R < a.M) {
+      row_range(a, L, R / a.G, slot_lo[i], slot_hi[i]);
+    } else {
+      slot_lo[i] = 0;
+      slot_hi[i] = 0;
+    }
+  }
+
+  float m_slot[C::NVF], l_slot[C::NVF];
+#pragma unroll
+  for (int i = 0; i < C::NVF; ++i) {
+    m_slot[i] = -INFINITY;
+    l_slot[i] = 0.f;
+  }
+  float acc[MT][8];
+#pragma unroll
+  for (int r = 0; r < MT; ++r)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
+
+  int n_fail = -1;  // tile whose copy never landed (bounded wait expired)
+
+  // ---- main loop over this warp's tiles -----------------------------------
+  for (int n = 0; n < my_tiles; ++n) {
+    const int s = n % STAGES;
+    if (!mbar_wait(&mbar[s], (n / STAGES) & 1, a.err)) {
+      n_fail = n;
+      break;
+    }
+    const uint8_t* kt = wbase + s * C::STAGE_BYTES;
+    const uint8_t* vt = kt + C::TILE_BYTES;
+    const int t0 = (kbase + n * NW) * TW;
+    const bool clean = t0 >= lo_x && t0 + TW <= hi_x;
+
+    // S = Q K^T, partial over this lane's 8 elements
+    float part[C::NV];
+#pragma unroll
+    for (int it = 0; it < C::NTOK; ++it) {
+      const int tok = it * C::TPI + grp;
+      float kf[8];
+      load_chunk<KV>(kt + (tok * D + d0) * C::ELT, kf);
+#pragma unroll
+      for (int r = 0; r < MT; ++r) {
+        float sacc = qf[r][0] * kf[0];
+#pragma unroll
+        for (int e = 1; e < 8; ++e) sacc = fmaf(qf[r][e], kf[e], sacc);
+        part[it * MT + r] = sacc;
+      }
+    }
+    // reduce-scatter over the LPT lanes of a token
+    reduce_scatter<C::NV, C::LPT / 2>(part, lane);
+    float sv[C::NVF];
+#pragma unroll
+    for (int i = 0; i < C::NVF; ++i) sv[i] = part[i];
+    if (!clean) {
+#pragma unroll
+      for (int i = 0; i < C::NVF; ++i) {
+        const int j = t0 + slot_tok[i];
+        if (!(j >= slot_lo[i] && j < slot_hi[i])) sv[i] = -INFINITY;
+      }
+    }
+
+    // tile row max over lanes holding the same rows
+    float rmax[C::NFOLD];
+#pragma unroll
+    for (int f = 0; f < C::NFOLD; ++f) {
+      rmax[f] = sv[f];
+#pragma unroll
+      for (int i = f + C::NFOLD; i < C::NVF; i += C::NFOLD) rmax[f] = fmaxf(rmax[f], sv[i]);
+    }
+#pragma unroll
+    for (int o = C::RED_LO; o < 32; o <<= 1)
+#pragma unroll
+      for (int f = 0; f < C::NFOLD; ++f)
+        rmax[f] = fmaxf(rmax[f], __shfl_xor_sync(FULL, rmax[f], o));
+
+    // online softmax update of the slots; p and alpha to shared memory
+#pragma unroll
+    for (int i = 0; i < C::NVF; ++i) {
+      const float m_new = fmaxf(m_slot[i], rmax[i % C::NFOLD]);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = fast_exp2(m_slot[i] - m_use);
+      const float p = fast_exp2(sv[i] - m_use);
+      l_slot[i] = l_slot[i] * alpha + p;
+      m_slot[i] = m_new;
+      pbuf[slot_tok[i] * MT + slot_row[i]] = p;
+      if (i < C::NFOLD) abuf[slot_row[i]] = alpha;
+    }
+    __syncwarp();
+
+    float al[MT];
+#pragma unroll
+    for (int r = 0; r < MT; ++r) al[r] = abuf[r];
+    bool rescale = false;
+#pragma unroll
+    for (int r = 0; r < MT; ++r) rescale |= al[r] != 1.f;
+    if (rescale) {
+#pragma unroll
+      for (int r = 0; r < MT; ++r)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[r][e] *= al[r];
+    }
+
+    // O += P V
+#pragma unroll
+    for (int it = 0; it < C::NTOK; ++it) {
+      const int tok = it * C::TPI + grp;
+      float pr[MT];
+      if constexpr (MT % 4 == 0) {
+#pragma unroll
+        for (int r = 0; r < MT; r += 4) {
+          const float4 p4 = *reinterpret_cast<const float4*>(pbuf + tok * MT + r);
+          pr[r] = p4.x; pr[r + 1] = p4.y; pr[r + 2] = p4.z; pr[r + 3] = p4.w;
+        }
+      } else if constexpr (MT == 2) {
+        const float2 p2 = *reinterpret_cast<const float2*>(pbuf + tok * MT);
+        pr[0] = p2.x; pr[1] = p2.y;
+      } else {
+        pr[0] = pbuf[tok];
+      }
+      float vf[8];
+      load_chunk<KV>(vt + (tok * D + d0) * C::ELT, vf);
+      if (!clean) {
+        const int j = t0 + tok;
+        if (j < lo_u || j >= hi_u) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) vf[e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < MT; ++r)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(pr[r], vf[e], acc[r][e]);
+    }
+    __syncwarp();
+    if (n + STAGES < my_tiles) {
+      if (lane == 0) fence_proxy_async_smem();
+      issue(n + STAGES);
+    }
+  }
+
+  if (n_fail >= 0) {
+    // Copies n_fail .. n_fail+STAGES-1 may still be in flight into this
+    // warp's ring: give each a short bounded wait before the memory is
+    // reused, so no copy lands in shared memory after the CTA has moved on.
+    const int issued = min(my_tiles, n_fail + STAGES);
+    for (int n = n_fail + 1; n < issued; ++n)
+      mbar_wait(&mbar[n % STAGES], (n / STAGES) & 1, a.err, kWaitTimeoutCycles / 8);
+  }
+
+  pdl_launch_dependents();
+
+  // ---- combine lane groups and rows inside the warp -----------------------
+#pragma unroll
+  for (int o = C::LPT; o < 32; o <<= 1)
+#pragma unroll
+    for (int r = 0; r < MT; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[r][e] += __shfl_xor_sync(FULL, acc[r][e], o);
+  float lsum[C::NFOLD];
+#pragma unroll
+  for (int f = 0; f < C::NFOLD; ++f) {
+    lsum[f] = l_slot[f];
+#pragma unroll
+    for (int i = f + C::NFOLD; i < C::NVF; i += C::NFOLD) lsum[f] += l_slot[i];
+  }
+#pragma unroll
+  for (int o = C::RED_LO; o < 32; o <<= 1)
+#pragma unroll
+    for (int f = 0; f < C::NFOLD; ++f) lsum[f] += __shfl_xor_sync(FULL, lsum[f], o);
+
+  // ---- merge the warps through shared memory -----------------------------
+  __syncthreads();  // every warp has drained its ring; stage memory is free
+  float* mrow = reinterpret_cast<float*>(smem);
+  float* lrow = mrow + NW * MT;
+  float* accs = lrow + NW * MT;
+#pragma unroll
+  for (int f = 0; f < C::NFOLD; ++f) {
+    mrow[warp * MT + slot_row[f]] = m_slot[f];
+    lrow[warp * MT + slot_row[f]] = lsum[f];
+  }
+  if (grp == 0) {
+#pragma unroll
+    for (int r = 0; r < MT; ++r) {
+      float4* dst = reinterpret_cast<float4*>(accs + (warp * MT + r) * D + d0);
+      dst[0] = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      dst[1] = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+    }
+  }
+  __syncthreads();
+
+  const long long rows_total = (long long)a.B * a.Lq * a.Hq;
+  for (int idx = threadIdx.x; idx < MT * (D / 4); idx += NW * 32) {
+    const int r = idx / (D / 4);
+    const int d = (idx % (D / 4)) * 4;
+    const int R = R0 + r;
+    if (R >= a.M) continue;
+    float mstar = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) mstar = fmaxf(mstar, mrow[w * MT + r]);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lt = 0.f;
+    if (mstar != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float wt = fast_exp2(mrow[w * MT + r] - mstar);
+        lt += wt * lrow[w * MT + r];
+        const float4 x = *reinterpret_cast<const float4*>(accs + (w * MT + r) * D + d);
+        o.x += wt * x.x; o.y += wt * x.y; o.z += wt * x.z; o.w += wt * x.w;
+      }
+    }
+    float res_lse = -INFINITY;
+    if (lt > 0.f) {
+      const float inv = a.v_scale / lt;
+      o.x *= inv; o.y *= inv; o.z *= inv; o.w *= inv;
+      res_lse = (mstar + log2f(lt)) * 0.69314718055994531f;
+    } else {
+      o = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int i = R / a.G, h = kvh * a.G + R % a.G;
+    const long long row = (long long)(b * a.Lq + i) * a.Hq + h;
+    if (a.num_splits == 1) {
+      *reinterpret_cast<float4*>(a.out + row * D + d) = o;
+      if (d == 0 && a.lse) a.lse[row] = res_lse;
+    } else {
+      const long long prow = (long long)split * rows_total + row;
+      *reinterpret_cast<float4*>(a.o_part + prow * D + d) = o;
+      if (d == 0) a.lse_part[prow] = res_lse;
+    }
+  }
+}
+
+// Host-side launcher for one head_dim, defined in split_d{64,128,256}.cu.
+// Returns cudaErrorNotSupported if no variant matches.
+cudaError_t launch_split_fma(int D, int kv, int mt, int tw, const SplitArgs& a,
+                             dim3 grid, cudaStream_t stream);
+
+}  // namespace pda

@@ -1,0 +1,70 @@
+// Instantiation and launch of the FMA split kernel variants for one head_dim.
+// Included by split_d64.cu / split_d128.cu / split_d256.cu, each compiled on
+// its own so the variants build in parallel.
+#pragma once
+
+#include "split_fma.cuh"
+
+namespace pda {
+
+// Warps per CTA and ring depth of each warp (one CTA per SM).
+constexpr int kFmaWarps = 8;
+constexpr int kFmaStages = 3;
+
+template <int D, int KV, int MT, int TW>
+cudaError_t launch_variant(const SplitArgs& a, dim3 grid, cudaStream_t stream) {
+  using C = FmaCfg<D, KV, MT, TW, kFmaWarps, kFmaStages>;
+  auto kern = split_fma_kernel<D, KV, MT, TW, kFmaWarps, kFmaStages>;
+  // The shared-memory opt-in is a per-device function attribute: set it the
+  // first time this variant launches on each device.
+  static unsigned long long attr_set = 0;  // bit d: set on device d (< 64)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit == 0 || !(__atomic_load_n(&attr_set, __ATOMIC_ACQUIRE) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
+  }
+  kern<<<grid, kFmaWarps * 32, C::SMEM, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int KV, int MT>
+cudaError_t launch_tw(int tw, const SplitArgs& a, dim3 grid, cudaStream_t s) {
+  constexpr int TW_FULL = 8 * (32 / (D / 8));  // 8 tokens per lane group
+  if (tw == TW_FULL) return launch_variant<D, KV, MT, TW_FULL>(a, grid, s);
+  if constexpr (TW_FULL / 2 >= 32 / (D / 8) && TW_FULL / 2 >= 8) {
+    if (tw == TW_FULL / 2) return launch_variant<D, KV, MT, TW_FULL / 2>(a, grid, s);
+  }
+  if constexpr (TW_FULL / 4 >= 32 / (D / 8) && TW_FULL / 4 >= 8) {
+    if (tw == TW_FULL / 4) return launch_variant<D, KV, MT, TW_FULL / 4>(a, grid, s);
+  }
+  return cudaErrorNotSupported;
+}
+
+template <int D>
+cudaError_t launch_for_dim(int kv, int mt, int tw, const SplitArgs& a,
+                           dim3 grid, cudaStream_t s) {
+#define PDA_MT_CASES(KV)                                      \
+  switch (mt) {                                               \
+    case 1: return launch_tw<D, KV, 1>(tw, a, grid, s);       \
+    case 2: return launch_tw<D, KV, 2>(tw, a, grid, s);       \
+    case 4: return launch_tw<D, KV, 4>(tw, a, grid, s);       \
+    case 8: return launch_tw<D, KV, 8>(tw, a, grid, s);       \
+    default: return cudaErrorNotSupported;                    \
+  }
+  if (kv == 0) {
+    PDA_MT_CASES(0)
+  } else {
+    PDA_MT_CASES(1)
+  }
+#undef PDA_MT_CASES
+}
+
+cudaError_t launch_split_d64(int kv, int mt, int tw, const SplitArgs& a, dim3 g, cudaStream_t s);
+cudaError_t launch_split_d128(int kv, int mt, int tw, const SplitArgs& a, dim3 g, cudaStream_t s);
+cudaError_t launch_split_d256(int kv, int mt, int tw, const SplitArgs& a, dim3 g, cudaStream_t s);
+
+}  // namespace pda

@@ -1,0 +1,161 @@
+"""The C-ABI library: loads, exports what the header declares, validates on the
+host (no GPU needed: every call here returns before any device work)."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from paged_kv_decode_30_b200 import binding as B
+from paged_kv_decode_30_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(
+                r"^\s*(?:PDA_API\s+)?(?:const\s+)?(?:pda_status|size_t|int32_t|char|void)\s*\**\s*(\w+)\s*\(",
+                text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_binding_surface():
+    assert declared_functions() == set(B.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_only_c_abi_symbols_are_exported(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    syms = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(B.EXPORTED) <= syms
+    assert not any(s.startswith("_ZN3pda") for s in syms), "C++ internals leaked"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.pda_abi_version() == 1
+    for code in range(8):
+        assert B.status_string(code)
+    assert B.status_string(99) == "unknown status"
+
+
+def headline_params(**over):
+    kw = dict(batch=128, q_len=1, num_q_heads=32, num_kv_heads=8, head_dim=128,
+              page_size=16, max_pages_per_seq=512, num_pages=65536,
+              scale=0.08838834764831845)
+    kw.update(over)
+    return B.make_params(**kw)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(head_dim=96), 2),
+    (dict(head_dim=0), 1),
+    (dict(page_size=12), 2),
+    (dict(page_size=4), 2),
+    (dict(page_size=512), 2),
+    (dict(q_len=0), 1),
+    (dict(q_len=9), 2),
+    (dict(num_q_heads=30), 1),
+    (dict(scale=0.0), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(causal_offset=-3), 1),
+    (dict(kv_dtype=2), 1),
+    (dict(kv_dtype=1, kv_scale=0.0), 1),
+    (dict(num_pages=0), 1),
+    (dict(max_pages_per_seq=0), 1),
+    (dict(num_splits=-1), 1),
+    (dict(batch=-1), 1),
+])
+def test_invalid_params_rejected_on_host(lib, over, status):
+    p = headline_params(**over)
+    dummy = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    st = lib.paged_decode_attn(dummy, dummy, dummy, dummy, dummy, ctypes.byref(p),
+                               dummy, dummy, None)
+    assert st == status, B.STATUS.get(st)
+
+
+def test_null_params_and_pointers(lib):
+    st = lib.paged_decode_attn(None, None, None, None, None, None, None, None, None)
+    assert st == 1
+    p = headline_params()
+    st = lib.paged_decode_attn(None, None, None, None, None, ctypes.byref(p), None, None, None)
+    assert st == 1
+
+
+def test_misaligned_pointers(lib):
+    p = headline_params()
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    st = lib.paged_decode_attn(bad, ok, ok, ok, ok, ctypes.byref(p), ok, ok, None)
+    assert st == 3
+    st = lib.paged_decode_attn(ok, ok, ok, ok, ok, ctypes.byref(p), bad, ok, None)
+    assert st == 3
+
+
+def test_empty_batch_is_a_no_op(lib):
+    p = headline_params(batch=0)
+    n = ctypes.c_int32(-5)
+    p.num_splits_out = ctypes.pointer(n)
+    st = lib.paged_decode_attn(None, None, None, None, None, ctypes.byref(p), None, None, None)
+    assert st == 0 and n.value == 1
+
+
+def test_merge_states_validation(lib):
+    st = lib.pda_merge_states(None, None, 0, 4, 128, None, None, None)
+    assert st == 1
+    st = lib.pda_merge_states(None, None, 2, 4, 96, None, None, None)
+    assert st == 2
+    st = lib.pda_merge_states(None, None, 2, 0, 128, None, None, None)
+    assert st == 0
+
+
+def test_split_planner(lib):
+    # headline: 1024 (b, kv head) units fill the 148 SMs ~7 times: no split
+    assert B.choose_num_splits(headline_params(), 148) == 1
+    # few long sequences: split to fill the machine
+    longctx = B.make_params(batch=4, q_len=1, num_q_heads=16, num_kv_heads=4,
+                            head_dim=256, page_size=128, max_pages_per_seq=256,
+                            num_pages=1024, scale=1 / 16)
+    s = B.choose_num_splits(longctx, 148)
+    assert 8 <= s <= 40, s
+    assert 16 * s <= 2 * 148
+    # forced split count is honoured (clamped to the tile count)
+    assert B.choose_num_splits(headline_params(num_splits=7), 148) == 7
+    tiny = B.make_params(batch=2, q_len=1, num_q_heads=4, num_kv_heads=1, head_dim=64,
+                         page_size=16, max_pages_per_seq=7, num_pages=16, scale=0.125)
+    assert B.choose_num_splits(tiny, 148) >= 1
+    assert B.choose_num_splits(B.make_params(
+        batch=2, q_len=1, num_q_heads=4, num_kv_heads=1, head_dim=64, page_size=16,
+        max_pages_per_seq=7, num_pages=16, scale=0.125, num_splits=1000), 148) <= 7
+    # the window bounds the span a CTA walks
+    win = headline_params(window=256, max_kv_len=8192, batch=4)
+    assert B.choose_num_splits(win, 148) <= 256 // 16
+
+
+def test_workspace_bytes(lib):
+    p = headline_params(num_splits=4)
+    rows = 128 * 32
+    expect_o = 4 * rows * 128 * 4
+    got = B.workspace_bytes(p)
+    assert got >= expect_o + 4 * rows * 4 and got < expect_o + 4 * rows * 4 + 512
+    assert B.workspace_bytes(headline_params(num_splits=1)) == 0
+    assert B.workspace_bytes(headline_params(head_dim=96)) == ctypes.c_size_t(-1).value

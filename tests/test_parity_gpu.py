@@ -1,0 +1,192 @@
+"""GPU parity: the CUDA library (through the C ABI) against the fp64 oracle on
+the same seeded inputs. Element by element on small and mid sizes spanning
+many tiles with ragged tails; sampled sequences at the full workload sizes."""
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_decode_30_b200 import binding as B
+from paged_kv_decode_30_b200 import workloads as W
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+BF16, FP8 = W.KV_BF16, W.KV_FP8_E4M3
+BR = W.CAUSAL_BOTTOM_RIGHT
+
+
+def wl(name, **kw):
+    base = dict(route="pool", seed=zlib.crc32(name.encode()) % 100000)
+    base.update(kw)
+    return W.Workload(name=name, **base)
+
+
+# Mid-size cases compared element by element.
+CASES = [
+    W.TINY,
+    wl("varlen_mid", batch=4, num_q_heads=32, num_kv_heads=8, head_dim=128, page_size=64,
+       kv_lens=("fixed", [1, 700, 64, 333]), extra_pages=5),
+    wl("headline_shape_bf16", batch=3, num_q_heads=32, num_kv_heads=8, head_dim=128,
+       page_size=16, kv_lens=("fixed", [1000, 517, 33]), extra_pages=3),
+    wl("headline_shape_fp8", batch=3, num_q_heads=32, num_kv_heads=8, head_dim=128,
+       page_size=16, kv_lens=("fixed", [1000, 517, 33]), extra_pages=3, kv_dtype=FP8),
+    wl("longctx_mid_peaked", batch=2, num_q_heads=16, num_kv_heads=4, head_dim=256,
+       page_size=128, scale=1 / 16, kv_lens=("fixed", [3000, 1111]), peaked_frac=0.01,
+       route="dense"),
+    wl("verify_fp8_window", batch=3, q_len=4, num_q_heads=64, num_kv_heads=8, head_dim=128,
+       page_size=128, kv_dtype=FP8, causal_offset=BR, window=512,
+       kv_lens=("fixed", [100, 700, 1500]), poison_invisible=True),
+    wl("verify_bf16_window", batch=3, q_len=4, num_q_heads=64, num_kv_heads=8, head_dim=128,
+       page_size=128, causal_offset=BR, window=512, kv_lens=("fixed", [100, 700, 1500]),
+       poison_invisible=True),
+    wl("d64_p8_mha", batch=3, num_q_heads=4, num_kv_heads=4, head_dim=64, page_size=8,
+       kv_lens=("fixed", [77, 8, 300])),
+    wl("d64_p256_gqa2_q3", batch=2, q_len=3, num_q_heads=4, num_kv_heads=2, head_dim=64,
+       page_size=256, causal_offset=BR, kv_lens=("fixed", [600, 2])),
+    wl("d128_p32_fixed_causal", batch=2, q_len=2, num_q_heads=8, num_kv_heads=1,
+       head_dim=128, page_size=32, causal_offset=100, kv_lens=("fixed", [300, 50])),
+    wl("d256_p16_window_noncausal", batch=2, num_q_heads=8, num_kv_heads=2, head_dim=256,
+       page_size=16, window=40, kv_lens=("fixed", [200, 39]), poison_invisible=True),
+    wl("empty_and_short_rows", batch=4, q_len=4, num_q_heads=8, num_kv_heads=2, head_dim=128,
+       page_size=16, causal_offset=BR, kv_lens=("fixed", [0, 1, 3, 20]), extra_pages=2),
+    wl("gqa8_q1_d128", batch=2, num_q_heads=16, num_kv_heads=2, head_dim=128, page_size=64,
+       kv_lens=("fixed", [900, 65])),
+    wl("fp8_d64_gqa4", batch=2, num_q_heads=8, num_kv_heads=2, head_dim=64, page_size=32,
+       kv_dtype=FP8, kv_lens=("fixed", [500, 31])),
+    wl("fp8_d256_q2", batch=2, q_len=2, num_q_heads=4, num_kv_heads=2, head_dim=256,
+       page_size=128, kv_dtype=FP8, causal_offset=BR, kv_lens=("fixed", [700, 129])),
+]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return B.load()
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("splits", [0, 1, 2, 3, 7, 64])
+def test_parity_vs_oracle(lib, case, splits):
+    inp = W.generate(case)
+    ref_out, ref_lse = U.run_oracle(inp)
+    out, lse, used = U.run_cuda(inp, num_splits=splits)
+    if splits:
+        assert 1 <= used <= splits
+    U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, f"{case.name}/s={splits}")
+
+
+@pytest.mark.parametrize("case", [CASES[2], CASES[5], CASES[7]], ids=lambda w: w.name)
+def test_page_permutation_invariance(lib, case):
+    inp = W.generate(case)
+    out0, lse0, _ = U.run_cuda(inp)
+    n = inp["k_pages"].shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(7))
+    k2 = torch.empty_like(inp["k_pages"])
+    v2 = torch.empty_like(inp["v_pages"])
+    k2[perm] = inp["k_pages"]
+    v2[perm] = inp["v_pages"]
+    pt = inp["page_table"].to(torch.int64)
+    pt2 = torch.where(pt >= 0, perm[pt.clamp(min=0)], pt).to(torch.int32)
+    out1, lse1, _ = U.run_cuda(dict(inp, k_pages=k2, v_pages=v2, page_table=pt2))
+    # the kernel's arithmetic depends only on logical token order
+    assert np.array_equal(out0, out1) and np.array_equal(lse0, lse1)
+
+
+def test_split_counts_agree_with_each_other(lib):
+    case = CASES[4]
+    inp = W.generate(case)
+    base_out, base_lse, _ = U.run_cuda(inp, num_splits=1)
+    for s in (2, 5, 9, 31):
+        out, lse, _ = U.run_cuda(inp, num_splits=s)
+        assert U.max_err(out, base_out) <= 1e-5
+        assert U.max_err(lse, base_lse) <= 1e-5
+
+
+def test_lse_may_be_null(lib):
+    inp = W.generate(CASES[2])
+    t = U.to_device(inp)
+    out, lse, _ = B.paged_decode_attn(
+        t["q"], t["k_pages"], t["v_pages"], t["page_table"], t["kv_lens"], num_kv_heads=8,
+        scale=W.scale_of(CASES[2]), with_lse=False, num_splits=3)
+    assert lse is None
+    ref_out, _ = U.run_oracle(inp)
+    assert U.max_err(out.double().cpu().numpy(), ref_out) <= 2e-3
+
+
+def test_merge_kernel_vs_oracle_merge(lib):
+    from oracle import oracle as orc
+    g = torch.Generator().manual_seed(3)
+    S, rows, D = 5, 300, 128
+    o = torch.randn((S, rows, D), generator=g, dtype=torch.float32)
+    ls = torch.randn((S, rows), generator=g, dtype=torch.float32) * 4
+    ls[1, ::3] = -float("inf")
+    o[1, ::3] = float("nan")          # never read when lse is -inf
+    ls[:, 7] = -float("inf")           # an empty row
+    o[:, 7] = float("nan")
+    out, lse = B.merge_states(o.cuda(), ls.cuda())
+    torch.cuda.synchronize()
+    o_ref = torch.where(torch.isnan(o), torch.zeros_like(o), o).double().numpy()
+    ref_out, ref_lse = orc.merge_states(o_ref, ls.double().numpy())
+    assert U.max_err(out.double().cpu().numpy(), ref_out) <= 1e-5
+    assert U.max_err(lse.double().cpu().numpy(), ref_lse) <= 1e-5
+
+
+def test_bad_page_id_is_reported_not_dereferenced(lib):
+    case = CASES[2]
+    inp = W.generate(case)
+    t = U.to_device(inp)
+    pt = t["page_table"].clone()
+    pt[1, 3] = inp["k_pages"].shape[0] + 1000   # outside the pool
+    pt[2, 0] = -7
+    B.last_device_error()
+    out, lse, _ = B.paged_decode_attn(
+        t["q"], t["k_pages"], t["v_pages"], pt, t["kv_lens"], num_kv_heads=8,
+        scale=W.scale_of(case))
+    assert B.last_device_error() == 6  # PDA_ERR_BAD_PAGE
+    assert B.last_device_error() == 0  # reading clears it
+    # sequence 0 never touched a bad page: still exact
+    ref_out, ref_lse = U.run_oracle(inp, seqs=[0])
+    U.assert_parity(out[:1].double().cpu().numpy(), lse[:1].double().cpu().numpy(),
+                    ref_out, ref_lse, BF16, "untouched sequence")
+
+
+def test_kv_len_beyond_page_table_is_reported(lib):
+    case = CASES[2]
+    inp = W.generate(case)
+    t = U.to_device(inp)
+    lens = t["kv_lens"].clone()
+    lens[0] = t["page_table"].shape[1] * case.page_size + 1
+    B.paged_decode_attn(t["q"], t["k_pages"], t["v_pages"], t["page_table"], lens,
+                        num_kv_heads=8, scale=W.scale_of(case))
+    assert B.last_device_error() == 6
+
+
+# ---------------------------------------------------------------------------
+# Full workload sizes, in the launch configuration the benchmark times.
+
+def _full(name):
+    return W.ALL[name]
+
+
+@pytest.mark.parametrize("name,seqs", [
+    (W.HEADLINE.name, [0, 57, 127]),
+    (W.FP8_VERIFY.name, [0, 1, 33, 63]),
+])
+def test_full_size_sampled(lib, name, seqs):
+    case = _full(name)
+    inp = W.generate(case, device="cuda")
+    out, lse, used = U.run_cuda(inp)
+    ref_out, ref_lse = U.run_oracle(inp, seqs=seqs)
+    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, case.kv_dtype, name)
+    assert np.isfinite(out).all()
+
+
+@pytest.mark.parametrize("name", [W.VARLEN.name, W.LONGCTX.name])
+def test_full_size_all_rows(lib, name):
+    case = _full(name)
+    inp = W.generate(case, device="cuda")
+    out, lse, used = U.run_cuda(inp)
+    ref_out, ref_lse = U.run_oracle(inp)
+    U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, name)
