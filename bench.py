@@ -45,6 +45,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0: planner)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (profiling a smaller case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -253,8 +255,10 @@ def run_reference(args, rank, world):
 def run_ours(args, rank, world, local):
     if not torch.cuda.is_available():
         raise RuntimeError("bench.py needs a CUDA device (the library has no CPU path)")
-    lib = B.load()
+    B.load()
     wl = W.ALL[args.workload]
+    if args.batch:
+        wl = wl.with_(batch=args.batch, name=f"{wl.name}_batch{args.batch}")
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = W.generate(wl, device=dev, seed=wl.seed + rank)
     scale = W.scale_of(wl)
