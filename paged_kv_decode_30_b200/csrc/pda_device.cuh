@@ -150,4 +150,46 @@ __device__ __forceinline__ void e4m3x8_to_f32(const uint2& u, float (&f)[8]) {
 
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
 
+// Two fp32 values in one 64-bit register pair, for the packed f32x2
+// arithmetic of sm_100 (one issue slot, two FMAs).
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// One 32-bit word holding two bf16 (element 2j in the low half, 2j+1 in the
+// high half) -> the fp32 pair (exact).
+__device__ __forceinline__ f32x2 bf16x2_to_f2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// Two e4m3 codes (16 bits) -> the fp32 pair (exact: e4m3 -> f16 -> f32).
+__device__ __forceinline__ f32x2 e4m3x2_to_f2(uint32_t h16) {
+  const __half2_raw hr =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(h16 & 0xFFFFu), __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+  return f2_pack(f.x, f.y);
+}
+
 }  // namespace pda

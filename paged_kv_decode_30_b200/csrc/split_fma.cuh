@@ -26,13 +26,18 @@
 //    for bf16, conflict-free). Q sits in registers, pre-scaled by
 //    scale*log2(e) (and kv_scale for FP8), for the lane's 8 elements of each
 //    of the M_T rows.
+//  * Arithmetic runs on packed fp32 pairs (fma/mul.rn.f32x2: two FMAs per
+//    issue slot); bf16 and e4m3 elements convert straight into pairs.
 //  * Scores: 8*M_T partial dot products per lane per group of 8 tokens are
 //    summed over the LPT lanes of a token with a reduce-scatter butterfly
 //    (each step halves the values a lane carries), so a score costs about one
-//    shuffle instead of log2(LPT).
+//    shuffle instead of log2(LPT). Each lane stores its partials in an order
+//    permuted by its own lane bits (it walks its tokens and its Q rows XORed
+//    with a lane mask), so that at every step all lanes keep the low half and
+//    send the high half: no selects.
 //  * Online softmax in fp32 with exp2; probabilities go through a small
-//    per-warp shared buffer to the P.V loop, which keeps acc[M_T][8] fp32 per
-//    lane.
+//    per-warp shared buffer (stored as (p, p) pairs) to the P.V loop, which
+//    keeps acc[M_T][8] fp32 per lane as pairs.
 //  * Masking by select, never by multiplying: scores of invisible keys become
 //    -inf; V of keys no row can see is zeroed before the FMA, so NaN bytes in
 //    tail slots or outside the window never reach the output. Tiles fully
@@ -83,9 +88,15 @@ struct FmaCfg {
       NV >= LPT ? (NVF >= MT ? 1 : MT / NVF) : (LPT / NV) * MT;
   static constexpr int TILE_BYTES = TW * D * ELT;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int PBUF_FLOATS = TW * MT;
+  static constexpr int PBUF_FLOATS = TW * MT * 2;  // (p, p) pairs
   static constexpr int WARP_SMEM_RAW =
-      STAGES * STAGE_BYTES + 32 /*mbarriers*/ + PBUF_FLOATS * 4 + 32 /*alpha*/;
+      STAGES * STAGE_BYTES + 32 /*mbarriers*/ + PBUF_FLOATS * 4 + 64 /*alpha pairs*/;
+  // lane-mask permutation of the reduce-scatter (see reduce_scatter)
+  static constexpr int LOG_LPT = LPT == 8 ? 3 : (LPT == 16 ? 4 : 5);
+  static constexpr int LOG_NV = NV == 1 ? 0 : NV == 2 ? 1 : NV == 4 ? 2 : NV == 8 ? 3 :
+                                NV == 16 ? 4 : NV == 32 ? 5 : NV == 64 ? 6 : 7;
+  static constexpr int LOG_MT = MT == 1 ? 0 : MT == 2 ? 1 : MT == 4 ? 2 : 3;
+  static constexpr int RS_STEPS = LOG_NV < LOG_LPT ? LOG_NV : LOG_LPT;
   static constexpr int WARP_SMEM = (WARP_SMEM_RAW + 127) / 128 * 128;
   static constexpr int MERGE_SMEM = (2 * NW * MT + NW * MT * D) * 4;
   static constexpr int SMEM =
@@ -116,37 +127,40 @@ __device__ __forceinline__ void row_range(const SplitArgs& a, int L, int i,
 }
 
 // Butterfly reduce-scatter of N values over the lanes whose ids differ in the
-// bits of O, O/2, ..., 1: at each step a lane keeps the half of its values
-// picked by its lane bit and adds the partner's copy of that half. After
-// log2(N) steps each lane holds one value summed over 2^(steps) lanes; the
+// bits of O, O/2, ..., 1. At each step every lane keeps v[0 .. N/2) and adds
+// the partner's v[N/2 .. N): the caller has stored its values permuted by its
+// lane mask, so that the low half of every lane is the half it must keep.
+// After log2(N) steps each lane holds one value summed over 2^steps lanes; the
 // remaining steps are plain butterflies. Values end in v[0 .. N/lanes).
 template <int N, int O>
-__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+__device__ __forceinline__ void reduce_scatter(float* v) {
   if constexpr (O >= 1) {
     if constexpr (N > 1) {
-      const bool up = (lane & O) != 0;
 #pragma unroll
-      for (int i = 0; i < N / 2; ++i) {
-        const float send = up ? v[i] : v[i + N / 2];
-        const float keep = up ? v[i + N / 2] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, O);
-      }
-      reduce_scatter<N / 2, O / 2>(v, lane);
+      for (int i = 0; i < N / 2; ++i) v[i] += __shfl_xor_sync(0xFFFFFFFFu, v[i + N / 2], O);
+      reduce_scatter<N / 2, O / 2>(v);
     } else {
       v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], O);
-      reduce_scatter<1, O / 2>(v, lane);
+      reduce_scatter<1, O / 2>(v);
     }
   }
 }
 
+// 8 consecutive K or V elements of one token -> 4 fp32 pairs.
 template <int KV>
-__device__ __forceinline__ void load_chunk(const uint8_t* p, float (&f)[8]) {
+__device__ __forceinline__ void load_chunk2(const uint8_t* p, f32x2 (&f)[4]) {
   if constexpr (KV == 0) {
     const uint4 u = *reinterpret_cast<const uint4*>(p);
-    bf16x8_to_f32(u, f);
+    f[0] = bf16x2_to_f2(u.x);
+    f[1] = bf16x2_to_f2(u.y);
+    f[2] = bf16x2_to_f2(u.z);
+    f[3] = bf16x2_to_f2(u.w);
   } else {
     const uint2 u = *reinterpret_cast<const uint2*>(p);
-    e4m3x8_to_f32(u, f);
+    f[0] = e4m3x2_to_f2(u.x);
+    f[1] = e4m3x2_to_f2(u.x >> 16);
+    f[2] = e4m3x2_to_f2(u.y);
+    f[3] = e4m3x2_to_f2(u.y >> 16);
   }
 }
 
@@ -240,33 +254,45 @@ __global__ void __launch_bounds__(NW * 32, 1)
   const int n_pro = my_tiles < STAGES ? my_tiles : STAGES;
   for (int n = 0; n < n_pro; ++n) issue(n);
 
-  // ---- Q fragment ----------------------------------------------------------
+  // ---- lane mask of the select-free reduce-scatter ------------------------
+  // The top RS_STEPS bits of the lane's chunk index c, placed as the top
+  // bits of the NV-value index: the lane stores value v at position
+  // v ^ vmask, i.e. walks tokens it ^ vmask_it and Q rows r ^ vmask_r.
   const int grp = lane / C::LPT;
-  const int d0 = (lane % C::LPT) * C::CH;
-  float qf[MT][8];
+  const int c = lane % C::LPT;
+  const int d0 = c * C::CH;
+  const int vmask = (c >> (C::LOG_LPT - C::RS_STEPS)) << (C::LOG_NV - C::RS_STEPS);
+  const int vmask_r = vmask & (MT - 1);
+  const int vmask_it = vmask >> C::LOG_MT;
+
+  // ---- Q fragment (rows permuted by vmask_r), as pairs ---------------------
+  f32x2 qf[MT][4];
+  {
+    const f32x2 sc = f2_pack(a.qk_scale_log2, a.qk_scale_log2);
 #pragma unroll
-  for (int r = 0; r < MT; ++r) {
-    const int R = R0 + r;
-    if (R < a.M) {
-      const int i = R / a.G, h = kvh * a.G + R % a.G;
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(
-          a.q + ((long long)(b * a.Lq + i) * a.Hq + h) * D + d0));
-      bf16x8_to_f32(u, qf[r]);
+    for (int r = 0; r < MT; ++r) {
+      const int R = R0 + (r ^ vmask_r);
+      if (R < a.M) {
+        const int i = R / a.G, h = kvh * a.G + R % a.G;
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+            a.q + ((long long)(b * a.Lq + i) * a.Hq + h) * D + d0));
+        qf[r][0] = f2_mul(bf16x2_to_f2(u.x), sc);
+        qf[r][1] = f2_mul(bf16x2_to_f2(u.y), sc);
+        qf[r][2] = f2_mul(bf16x2_to_f2(u.z), sc);
+        qf[r][3] = f2_mul(bf16x2_to_f2(u.w), sc);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qf[r][e] *= a.qk_scale_log2;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qf[r][e] = 0.f;
+        for (int j = 0; j < 4; ++j) qf[r][j] = 0ull;
+      }
     }
   }
 
   // ---- slots this lane holds after the reduce-scatter --------------------
-  const int c = lane % C::LPT;
-  const int vbase = C::NV >= C::LPT ? c * C::NVF : c / (C::LPT / C::NV);
+  // slot i holds value v = vmask | i: token (v / MT) * TPI + grp, row v % MT
   int slot_tok[C::NVF], slot_row[C::NVF], slot_lo[C::NVF], slot_hi[C::NVF];
 #pragma unroll
   for (int i = 0; i < C::NVF; ++i) {
-    const int v = vbase + i;
+    const int v = vmask | i;
     slot_tok[i] = (v / MT) * C::TPI + grp;
     slot_row[i] = v % MT;
     const int R = R0 + slot_row[i];
@@ -284,11 +310,11 @@ __global__ void __launch_bounds__(NW * 32, 1)
     m_slot[i] = -INFINITY;
     l_slot[i] = 0.f;
   }
-  float acc[MT][8];
+  f32x2 acc[MT][4];
 #pragma unroll
   for (int r = 0; r < MT; ++r)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[r][j] = 0ull;  // (+0.f, +0.f)
 
   int n_fail = -1;  // tile whose copy never landed (bounded wait expired)
 
@@ -304,23 +330,25 @@ __global__ void __launch_bounds__(NW * 32, 1)
     const int t0 = (kbase + n * NW) * TW;
     const bool clean = t0 >= lo_x && t0 + TW <= hi_x;
 
-    // S = Q K^T, partial over this lane's 8 elements
+    // S = Q K^T, partial over this lane's 8 elements, stored permuted
     float part[C::NV];
 #pragma unroll
     for (int it = 0; it < C::NTOK; ++it) {
-      const int tok = it * C::TPI + grp;
-      float kf[8];
-      load_chunk<KV>(kt + (tok * D + d0) * C::ELT, kf);
+      const int tok = (it ^ vmask_it) * C::TPI + grp;
+      f32x2 kf[4];
+      load_chunk2<KV>(kt + (tok * D + d0) * C::ELT, kf);
 #pragma unroll
       for (int r = 0; r < MT; ++r) {
-        float sacc = qf[r][0] * kf[0];
-#pragma unroll
-        for (int e = 1; e < 8; ++e) sacc = fmaf(qf[r][e], kf[e], sacc);
-        part[it * MT + r] = sacc;
+        f32x2 s2 = f2_mul(qf[r][0], kf[0]);
+        s2 = f2_fma(qf[r][1], kf[1], s2);
+        s2 = f2_fma(qf[r][2], kf[2], s2);
+        s2 = f2_fma(qf[r][3], kf[3], s2);
+        float lo, hi;
+        f2_unpack(s2, lo, hi);
+        part[it * MT + r] = lo + hi;
       }
     }
-    // reduce-scatter over the LPT lanes of a token
-    reduce_scatter<C::NV, C::LPT / 2>(part, lane);
+    reduce_scatter<C::NV, C::LPT / 2>(part);
     float sv[C::NVF];
 #pragma unroll
     for (int i = 0; i < C::NVF; ++i) sv[i] = part[i];
@@ -346,7 +374,8 @@ __global__ void __launch_bounds__(NW * 32, 1)
       for (int f = 0; f < C::NFOLD; ++f)
         rmax[f] = fmaxf(rmax[f], __shfl_xor_sync(FULL, rmax[f], o));
 
-    // online softmax update of the slots; p and alpha to shared memory
+    // online softmax update of the slots; (p, p) and (alpha, alpha) pairs to
+    // shared memory
 #pragma unroll
     for (int i = 0; i < C::NVF; ++i) {
       const float m_new = fmaxf(m_slot[i], rmax[i % C::NFOLD]);
@@ -355,54 +384,58 @@ __global__ void __launch_bounds__(NW * 32, 1)
       const float p = fast_exp2(sv[i] - m_use);
       l_slot[i] = l_slot[i] * alpha + p;
       m_slot[i] = m_new;
-      pbuf[slot_tok[i] * MT + slot_row[i]] = p;
-      if (i < C::NFOLD) abuf[slot_row[i]] = alpha;
+      reinterpret_cast<float2*>(pbuf)[slot_tok[i] * MT + slot_row[i]] = make_float2(p, p);
+      if (i < C::NFOLD) reinterpret_cast<float2*>(abuf)[slot_row[i]] = make_float2(alpha, alpha);
     }
     __syncwarp();
 
-    float al[MT];
+    {
+      f32x2 al[MT];
+      bool rescale = false;
 #pragma unroll
-    for (int r = 0; r < MT; ++r) al[r] = abuf[r];
-    bool rescale = false;
+      for (int r = 0; r < MT; ++r) {
+        const float2 x = reinterpret_cast<const float2*>(abuf)[r];
+        al[r] = f2_pack(x.x, x.y);
+        rescale |= x.x != 1.f;
+      }
+      if (rescale) {
 #pragma unroll
-    for (int r = 0; r < MT; ++r) rescale |= al[r] != 1.f;
-    if (rescale) {
+        for (int r = 0; r < MT; ++r)
 #pragma unroll
-      for (int r = 0; r < MT; ++r)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][e] *= al[r];
+          for (int j = 0; j < 4; ++j) acc[r][j] = f2_mul(acc[r][j], al[r]);
+      }
     }
 
     // O += P V
 #pragma unroll
     for (int it = 0; it < C::NTOK; ++it) {
       const int tok = it * C::TPI + grp;
-      float pr[MT];
-      if constexpr (MT % 4 == 0) {
+      f32x2 pr[MT];
+      const float4* pp = reinterpret_cast<const float4*>(pbuf + tok * MT * 2);
+      if constexpr (MT >= 2) {
 #pragma unroll
-        for (int r = 0; r < MT; r += 4) {
-          const float4 p4 = *reinterpret_cast<const float4*>(pbuf + tok * MT + r);
-          pr[r] = p4.x; pr[r + 1] = p4.y; pr[r + 2] = p4.z; pr[r + 3] = p4.w;
+        for (int r = 0; r < MT; r += 2) {
+          const float4 p4 = pp[r / 2];
+          pr[r] = f2_pack(p4.x, p4.y);
+          pr[r + 1] = f2_pack(p4.z, p4.w);
         }
-      } else if constexpr (MT == 2) {
-        const float2 p2 = *reinterpret_cast<const float2*>(pbuf + tok * MT);
-        pr[0] = p2.x; pr[1] = p2.y;
       } else {
-        pr[0] = pbuf[tok];
+        const float2 p2 = reinterpret_cast<const float2*>(pbuf)[tok];
+        pr[0] = f2_pack(p2.x, p2.y);
       }
-      float vf[8];
-      load_chunk<KV>(vt + (tok * D + d0) * C::ELT, vf);
+      f32x2 vf[4];
+      load_chunk2<KV>(vt + (tok * D + d0) * C::ELT, vf);
       if (!clean) {
         const int j = t0 + tok;
         if (j < lo_u || j >= hi_u) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) vf[e] = 0.f;
+          for (int e = 0; e < 4; ++e) vf[e] = 0ull;
         }
       }
 #pragma unroll
       for (int r = 0; r < MT; ++r)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(pr[r], vf[e], acc[r][e]);
+        for (int e = 0; e < 4; ++e) acc[r][e] = f2_fma(pr[r], vf[e], acc[r][e]);
     }
     __syncwarp();
     if (n + STAGES < my_tiles) {
@@ -423,12 +456,17 @@ __global__ void __launch_bounds__(NW * 32, 1)
   pdl_launch_dependents();
 
   // ---- combine lane groups and rows inside the warp -----------------------
+  float accf[MT][8];
+#pragma unroll
+  for (int r = 0; r < MT; ++r)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) f2_unpack(acc[r][j], accf[r][2 * j], accf[r][2 * j + 1]);
 #pragma unroll
   for (int o = C::LPT; o < 32; o <<= 1)
 #pragma unroll
     for (int r = 0; r < MT; ++r)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[r][e] += __shfl_xor_sync(FULL, acc[r][e], o);
+      for (int e = 0; e < 8; ++e) accf[r][e] += __shfl_xor_sync(FULL, accf[r][e], o);
   float lsum[C::NFOLD];
 #pragma unroll
   for (int f = 0; f < C::NFOLD; ++f) {
@@ -455,8 +493,8 @@ __global__ void __launch_bounds__(NW * 32, 1)
 #pragma unroll
     for (int r = 0; r < MT; ++r) {
       float4* dst = reinterpret_cast<float4*>(accs + (warp * MT + r) * D + d0);
-      dst[0] = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-      dst[1] = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+      dst[0] = make_float4(accf[r][0], accf[r][1], accf[r][2], accf[r][3]);
+      dst[1] = make_float4(accf[r][4], accf[r][5], accf[r][6], accf[r][7]);
     }
   }
   __syncthreads();
