@@ -109,7 +109,7 @@ Plan make_plan(const pda_params* p) {
   pl.tw = p->page_size < tw_full ? p->page_size : tw_full;
   pl.elt = p->kv_dtype == PDA_KV_BF16 ? 2 : 1;
   pl.rows = (long long)p->batch * p->q_len * p->num_q_heads;
-  pl.tiles_per_cta_iter = pl.tw * kFmaWarps;
+  pl.tiles_per_cta_iter = pl.tw * fma_warps(pl.mt);
   return pl;
 }
 

@@ -7,14 +7,24 @@
 
 namespace pda {
 
-// Warps per CTA and ring depth of each warp (one CTA per SM).
-constexpr int kFmaWarps = 8;
-constexpr int kFmaStages = 3;
+// Warps per CTA and ring depth of each warp (one CTA per SM). The kernel is
+// bound by issue latency, not by bytes in flight: 12 warps with a 2-deep
+// ring (3 warps per scheduler, 168 registers) beat 8 warps with a 3-deep
+// ring by 13% on the headline shape. Variants with 8 packed rows need more
+// than 168 registers, so they keep 8 warps x 3 stages.
+template <int MT>
+struct FmaShape {
+  static constexpr int NW = MT <= 4 ? 12 : 8;
+  static constexpr int STAGES = MT <= 4 ? 2 : 3;
+};
+inline int fma_warps(int mt) { return mt <= 4 ? 12 : 8; }
 
 template <int D, int KV, int MT, int TW>
 cudaError_t launch_variant(const SplitArgs& a, dim3 grid, cudaStream_t stream) {
-  using C = FmaCfg<D, KV, MT, TW, kFmaWarps, kFmaStages>;
-  auto kern = split_fma_kernel<D, KV, MT, TW, kFmaWarps, kFmaStages>;
+  constexpr int NW = FmaShape<MT>::NW;
+  constexpr int ST = FmaShape<MT>::STAGES;
+  using C = FmaCfg<D, KV, MT, TW, NW, ST>;
+  auto kern = split_fma_kernel<D, KV, MT, TW, NW, ST>;
   // The shared-memory opt-in is a per-device function attribute: set it the
   // first time this variant launches on each device.
   static unsigned long long attr_set = 0;  // bit d: set on device d (< 64)
@@ -27,7 +37,7 @@ cudaError_t launch_variant(const SplitArgs& a, dim3 grid, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
   }
-  kern<<<grid, kFmaWarps * 32, C::SMEM, stream>>>(a);
+  kern<<<grid, NW * 32, C::SMEM, stream>>>(a);
   return cudaGetLastError();
 }
 
