@@ -140,6 +140,43 @@ PDA_API pda_status paged_decode_attn(const void* q, const void* k_pages,
                              const int32_t* kv_lens, const pda_params* params,
                              float* out, float* lse, pda_stream_t stream);
 
+/*
+ * paged_decode_attn for callers that cannot allocate device memory. The
+ * pages describe no counterpart to this entry point; it exists for callers
+ * such as a serving engine that reserves nearly all of HBM for its own
+ * KV-cache pool at start-up and forbids later allocations, or code on a
+ * latency-critical path where cudaMalloc / cudaFree may synchronise the
+ * device, and that cannot hand the library a workspace either.
+ *
+ * Same arguments and results as paged_decode_attn, except that
+ * params->workspace and params->workspace_bytes are ignored: the split-KV
+ * partials live in a fixed array of PDA_NO_ALLOC_WORKSPACE_BYTES compiled
+ * into the library, which every device that loads the library holds until
+ * the process exits. The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *
+ * Limit: if the partials of the chosen (or forced) split count need more
+ * than PDA_NO_ALLOC_WORKSPACE_BYTES (see paged_decode_attn_workspace_bytes),
+ * the call returns PDA_ERR_WORKSPACE before any device work.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.
+ *
+ * Sharing: all calls on a device use the same array, which keeps the last
+ * call's partials. Nothing in it needs clearing (every slot a call reads was
+ * written earlier in that call), but calls that overlap on the GPU (on
+ * different streams) race on it: serialise them.
+ */
+#define PDA_NO_ALLOC_WORKSPACE_BYTES (16u * 1024u * 1024u)
+
+PDA_API pda_status paged_decode_attn_no_alloc(const void* q, const void* k_pages,
+                                              const void* v_pages,
+                                              const int32_t* page_table,
+                                              const int32_t* kv_lens,
+                                              const pda_params* params, float* out,
+                                              float* lse, pda_stream_t stream);
+
 /* Bytes of workspace paged_decode_attn needs for these params with the
  * split count it would choose (0 when it would not split). SIZE_MAX if the
  * params are invalid. */

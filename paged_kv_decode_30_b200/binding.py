@@ -20,6 +20,8 @@ PDA_KV_FP8_E4M3 = 1
 PDA_CAUSAL_OFF = -1
 PDA_CAUSAL_BOTTOM_RIGHT = -2
 PDA_FLAG_NO_PDL = 1
+# Size of the library's fixed partials array used by paged_decode_attn_no_alloc.
+PDA_NO_ALLOC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 STATUS = {
     0: "PDA_OK", 1: "PDA_ERR_INVALID_ARG", 2: "PDA_ERR_UNSUPPORTED",
@@ -29,7 +31,7 @@ STATUS = {
 
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTED = (
-    "paged_decode_attn", "paged_decode_attn_workspace_bytes",
+    "paged_decode_attn", "paged_decode_attn_no_alloc", "paged_decode_attn_workspace_bytes",
     "pda_choose_num_splits", "pda_merge_states", "pda_status_string",
     "pda_last_device_error", "pda_abi_version",
 )
@@ -85,6 +87,8 @@ def load(path: Optional[str] = None):
     pp = ctypes.POINTER(PdaParams)
     lib.paged_decode_attn.restype = i32
     lib.paged_decode_attn.argtypes = [vp, vp, vp, vp, vp, pp, vp, vp, vp]
+    lib.paged_decode_attn_no_alloc.restype = i32
+    lib.paged_decode_attn_no_alloc.argtypes = [vp, vp, vp, vp, vp, pp, vp, vp, vp]
     lib.paged_decode_attn_workspace_bytes.restype = ctypes.c_size_t
     lib.paged_decode_attn_workspace_bytes.argtypes = [pp]
     lib.pda_choose_num_splits.restype = i32
@@ -186,6 +190,37 @@ def paged_decode_attn(q, k_pages, v_pages, page_table, kv_lens, *, num_kv_heads,
         ctypes.byref(params), _ptr(out), _ptr(lse), _stream_handle(stream))
     if st != 0:
         raise PdaError(st, "paged_decode_attn")
+    return out, lse, used.value
+
+
+def paged_decode_attn_no_alloc(q, k_pages, v_pages, page_table, kv_lens, *,
+                               num_kv_heads, scale, causal_offset=PDA_CAUSAL_OFF,
+                               window=0, kv_scale=1.0, max_kv_len=0, num_splits=0,
+                               flags=0, out=None, lse=None, stream=None):
+    """The allocation-free entry point: split partials go to the library's
+    fixed device array instead of a workspace (see the C header). ``out`` and
+    ``lse`` are allocated here by torch only when the caller passes None."""
+    import torch
+    lib = load()
+    B, q_len, Hq, D = q.shape
+    kv_dtype = PDA_KV_FP8_E4M3 if k_pages.dtype == torch.uint8 else PDA_KV_BF16
+    params = make_params(
+        batch=B, q_len=q_len, num_q_heads=Hq, num_kv_heads=num_kv_heads, head_dim=D,
+        page_size=k_pages.shape[2], max_pages_per_seq=page_table.shape[1],
+        num_pages=k_pages.shape[0], scale=scale, causal_offset=causal_offset,
+        window=window, kv_dtype=kv_dtype, kv_scale=kv_scale, max_kv_len=max_kv_len,
+        num_splits=num_splits, flags=flags)
+    if out is None:
+        out = torch.empty((B, q_len, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, q_len, Hq), dtype=torch.float32, device=q.device)
+    used = ctypes.c_int32(0)
+    params.num_splits_out = ctypes.pointer(used)
+    st = lib.paged_decode_attn_no_alloc(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(kv_lens),
+        ctypes.byref(params), _ptr(out), _ptr(lse), _stream_handle(stream))
+    if st != 0:
+        raise PdaError(st, "paged_decode_attn_no_alloc")
     return out, lse, used.value
 
 
