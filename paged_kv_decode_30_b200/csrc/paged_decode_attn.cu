@@ -16,6 +16,7 @@
 
 #include "merge.cuh"
 #include "paged_decode_attn.h"
+#include "split_tc.cuh"
 #include "split_variants.cuh"
 
 namespace pda {
@@ -75,7 +76,15 @@ struct Plan {
   int G, M, mt, row_tiles, tw, elt;
   long long rows;          // B * q_len * Hq
   int tiles_per_cta_iter;  // tokens one CTA iteration covers = tw * warps
+  bool tc;                 // tensor-core kernel (else the FMA kernel)
 };
+
+// The tensor-core kernel takes FP8 K/V with head_dim 128 when the packed
+// rows of a kv head (G * q_len) exceed what the FMA kernel holds in one CTA
+// (8): then QK^T and PV are real dense contractions (N = 16 or 32 rows).
+bool use_tensor_cores(const pda_params* p, int M) {
+  return p->kv_dtype == PDA_KV_FP8_E4M3 && p->head_dim == 128 && M > 8 && p->page_size >= 8;
+}
 
 pda_status validate(const pda_params* p) {
   if (p == nullptr) return PDA_ERR_INVALID_ARG;
@@ -103,13 +112,20 @@ Plan make_plan(const pda_params* p) {
   Plan pl{};
   pl.G = p->num_q_heads / p->num_kv_heads;
   pl.M = pl.G * p->q_len;
-  pl.mt = pl.M >= 8 ? 8 : (pl.M >= 4 ? 4 : (pl.M >= 2 ? 2 : 1));
-  pl.row_tiles = (int)cdiv(pl.M, pl.mt);
-  const int tw_full = 8 * (32 / (p->head_dim / 8));
-  pl.tw = p->page_size < tw_full ? p->page_size : tw_full;
   pl.elt = p->kv_dtype == PDA_KV_BF16 ? 2 : 1;
   pl.rows = (long long)p->batch * p->q_len * p->num_q_heads;
-  pl.tiles_per_cta_iter = pl.tw * fma_warps(pl.mt);
+  pl.tc = use_tensor_cores(p, pl.M);
+  if (pl.tc) {
+    pl.mt = pl.M <= 16 ? 16 : 32;  // rows per CTA (MMA N)
+    pl.tw = 128;                   // tokens per tile (MMA M)
+    pl.tiles_per_cta_iter = 128;
+  } else {
+    pl.mt = pl.M >= 8 ? 8 : (pl.M >= 4 ? 4 : (pl.M >= 2 ? 2 : 1));
+    const int tw_full = 8 * (32 / (p->head_dim / 8));
+    pl.tw = p->page_size < tw_full ? p->page_size : tw_full;
+    pl.tiles_per_cta_iter = pl.tw * fma_warps(pl.mt);
+  }
+  pl.row_tiles = (int)cdiv(pl.M, pl.mt);
   return pl;
 }
 
@@ -254,7 +270,7 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   a.log2_page = ilog2(p.page_size);
   a.max_pages = p.max_pages_per_seq;
   a.num_pages = p.num_pages;
-  a.tile_shift = ilog2(p.page_size / pl.tw);
+  a.tile_shift = pl.tc ? 0 : ilog2(p.page_size / pl.tw);
   a.num_splits = splits;
   a.row_tiles = pl.row_tiles;
   a.causal_offset = p.causal_offset;
@@ -293,7 +309,9 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   const dim3 grid((unsigned)pl.row_tiles, (unsigned)(splits * p.num_kv_heads), (unsigned)p.batch);
   cudaError_t e;
   const int kv = fp8 ? 1 : 0;
-  switch (p.head_dim) {
+  if (pl.tc) {
+    e = launch_split_tc(pl.mt, a, grid, stream);
+  } else switch (p.head_dim) {
     case 64: e = launch_split_d64(kv, pl.mt, pl.tw, a, grid, stream); break;
     case 128: e = launch_split_d128(kv, pl.mt, pl.tw, a, grid, stream); break;
     case 256: e = launch_split_d256(kv, pl.mt, pl.tw, a, grid, stream); break;

@@ -58,6 +58,18 @@ CASES = [
        kv_dtype=FP8, kv_lens=("fixed", [500, 31])),
     wl("fp8_d256_q2", batch=2, q_len=2, num_q_heads=4, num_kv_heads=2, head_dim=256,
        page_size=128, kv_dtype=FP8, causal_offset=BR, kv_lens=("fixed", [700, 129])),
+    # tensor-core path: FP8, head_dim 128, more than 8 packed rows per kv head
+    wl("tc_fp8_p16_q2_g8", batch=4, q_len=2, num_q_heads=16, num_kv_heads=2, head_dim=128,
+       page_size=16, kv_dtype=FP8, causal_offset=BR, kv_lens=("fixed", [1, 130, 1000, 2047]),
+       extra_pages=4),
+    wl("tc_fp8_p256_g16", batch=2, num_q_heads=32, num_kv_heads=2, head_dim=128,
+       page_size=256, kv_dtype=FP8, kv_lens=("fixed", [300, 5000])),
+    wl("tc_fp8_p64_q3_g16_window", batch=3, q_len=3, num_q_heads=32, num_kv_heads=2,
+       head_dim=128, page_size=64, kv_dtype=FP8, causal_offset=BR, window=200,
+       kv_lens=("fixed", [2, 333, 1500]), poison_invisible=True),
+    wl("tc_fp8_fixed_offset_empty", batch=3, q_len=4, num_q_heads=64, num_kv_heads=8,
+       head_dim=128, page_size=128, kv_dtype=FP8, causal_offset=40, window=30,
+       kv_lens=("fixed", [0, 20, 700]), extra_pages=2),
 ]
 
 
