@@ -209,8 +209,10 @@ PDA_API pda_status pda_merge_states(const float* o_parts, const float* lse_parts
 PDA_API const char* pda_status_string(pda_status status);
 
 /* Synchronises `stream`, then reads and clears the current device's error
- * word: PDA_ERR_BAD_PAGE or PDA_ERR_TIMEOUT if a kernel recorded one since
- * the last read, PDA_OK otherwise (PDA_ERR_CUDA if the sync failed). */
+ * word: the first error a kernel recorded since the last read
+ * (PDA_ERR_BAD_PAGE, PDA_ERR_TIMEOUT, or PDA_ERR_UNSUPPORTED if a kernel met
+ * a launch condition it cannot handle), PDA_OK otherwise (PDA_ERR_CUDA if the
+ * sync failed). */
 PDA_API pda_status pda_last_device_error(pda_stream_t stream);
 
 /* PDA_ABI_VERSION of the loaded library. */

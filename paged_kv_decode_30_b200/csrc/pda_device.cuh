@@ -15,6 +15,7 @@
 
 namespace pda {
 
+constexpr int kErrUnsupported = 2;  // == PDA_ERR_UNSUPPORTED
 constexpr int kErrBadPage = 6;   // == PDA_ERR_BAD_PAGE
 constexpr int kErrTimeout = 7;   // == PDA_ERR_TIMEOUT
 

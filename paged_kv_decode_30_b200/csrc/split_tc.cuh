@@ -53,8 +53,18 @@ struct TcCfg {
   static constexpr int RAW_STAGE = 2 * RAW_TILE;     // K + V
   static constexpr int OP_TILE = TILE * D * 2;       // one f16 K (or V) operand tile
   static constexpr int Q_BYTES = NT * D * 2;
-  static constexpr int P_LBO = (NT / 8) * 128;       // P^T: token-group stride
-  static constexpr int P_BYTES = (TILE / 8) * P_LBO;
+  // K, V (tokens x head_dim) and Q (rows x head_dim) share one physical
+  // layout: two 64-element halves of head_dim, each a column of SW128 atoms
+  // (8 rows x 128 B), atom g of rows 8g..8g+7 at g*1024. The same bytes are
+  // the K-major operand K (S^T = K Q^T) and the MN-major operand V^T.
+  static constexpr int KV_HALF = (TILE / 8) * 1024;  // one 64-element half
+  static constexpr int Q_HALF = (NT / 8) * 1024;
+  // P^T (rows x tokens, rows contiguous): one atom of 8 tokens x NT rows,
+  // SW64 (NT = 32, 64-byte rows) or SW32 (NT = 16, 32-byte rows)
+  static constexpr int P_ROW = NT * 2;               // bytes per token row
+  static constexpr int P_SBO = 8 * P_ROW;            // token-group stride
+  static constexpr int P_BYTES = (TILE / 8) * P_SBO;
+  static constexpr uint32_t P_SWIZZLE = NT == 32 ? 4u : 6u;  // SW64 / SW32
   // shared memory map
   static constexpr int OFF_RAW = 0;
   static constexpr int OFF_K = OFF_RAW + RAW_STAGES * RAW_STAGE;
@@ -81,22 +91,41 @@ struct TcCfg {
   static_assert(NT == 16 || NT == 32, "rows per CTA");
   static_assert(4 * NT <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
-  static_assert(OFF_K % 1024 == 0 && OFF_Q % 128 == 0 && OFF_P % 128 == 0, "alignment");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_Q % 1024 == 0 &&
+                    OFF_P % 1024 == 0 && P_BYTES % 1024 == 0,
+                "swizzle atoms need 1024-byte aligned bases");
 };
 
 // ---- tcgen05 / UMMA helpers ------------------------------------------------
 
-// Shared-memory matrix descriptor, no swizzle (canonical "interleaved"
-// layout of 8-row x 16-byte core matrices): start address, leading-dimension
-// byte offset (between core matrices along K for K-major operands, along the
-// K groups for MN-major ones) and stride-dimension byte offset.
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor: start address, leading- and stride-
+// dimension byte offsets, and the swizzle mode of the canonical layout.
+// Swizzled atoms are 8 rows of 128 (SW128), 64 (SW64) or 32 (SW32) bytes
+// whose 16-byte chunks are XOR-permuted by row, which keeps the tensor
+// core's operand reads free of bank conflicts. Atom bases are aligned to
+// 8 rows x row bytes, so the base-offset field stays 0.
+constexpr uint32_t kSw128 = 2, kSw64 = 4, kSw32 = 6;
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;  // descriptor version for sm_100
-  return d;                // base offset 0, layout type 0 (no swizzle)
+  d |= (uint64_t)(layout & 7u) << 61;
+  return d;
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: f16 A and B, fp32 D.
@@ -268,8 +297,13 @@ __global__ void __launch_bounds__(TcCfg<NT>::THREADS, 1) split_tc_kernel(const S
   const int n_all = k_end - k_begin;
   const int chunk = (n_all + a.num_splits - 1) / a.num_splits;
   const int c0 = min(n_all, split * chunk);
-  const int ntiles = min(n_all, c0 + chunk) - c0;
+  int ntiles = min(n_all, c0 + chunk) - c0;
   const int kfirst = k_begin + c0;
+  // The swizzle patterns below assume 1024-byte aligned atoms.
+  if ((smem_addr(smem) & 1023u) != 0) {
+    if (tid == 0) record_error_at(a.err, kErrUnsupported);
+    ntiles = 0;
+  }
 
   if (tid == 0) {
 #pragma unroll
@@ -347,7 +381,7 @@ __global__ void __launch_bounds__(TcCfg<NT>::THREADS, 1) split_tc_kernel(const S
     const int t = tid;  // 0..127
     // Q (rows R0 .. R0+NT-1) -> f16, K-major canonical layout; row >= M -> 0
     for (int c = t; c < NT * 16; c += 128) {
-      const int n = c >> 4, j = c & 15;
+      const int n = c % NT, j = c / NT;  // row, 8-element chunk of head_dim
       const int R = R0 + n;
       uint4 o = make_uint4(0, 0, 0, 0);
       if (R < a.M) {
@@ -361,7 +395,8 @@ __global__ void __launch_bounds__(TcCfg<NT>::THREADS, 1) split_tc_kernel(const S
         o.z = pack_f16x2(f[4], f[5]);
         o.w = pack_f16x2(f[6], f[7]);
       }
-      *reinterpret_cast<uint4*>(smem + C::OFF_Q + (n >> 3) * 2048 + j * 128 + (n & 7) * 16) = o;
+      *reinterpret_cast<uint4*>(smem + C::OFF_Q + (j >> 3) * C::Q_HALF + (n >> 3) * 1024 +
+                                (n & 7) * 128 + (((j & 7) ^ (n & 7)) << 4)) = o;
     }
     int issued = 0;  // tiles whose copies thread 0 has issued
     if (t == 0) {
@@ -401,15 +436,17 @@ __global__ void __launch_bounds__(TcCfg<NT>::THREADS, 1) split_tc_kernel(const S
       }
       const int j_tok = (kfirst + n) * C::TILE + t;
       const bool v_zero = j_tok < lo_u || j_tok >= hi_u;
-      uint8_t* sk = smem + C::OFF_K + bb * C::OP_TILE + (t >> 3) * 2048 + (t & 7) * 16;
-      uint8_t* sv = smem + C::OFF_V + bb * C::OP_TILE + (t >> 3) * 2048 + (t & 7) * 16;
+      const int row_off = (t >> 3) * 1024 + (t & 7) * 128;
+      uint8_t* sk = smem + C::OFF_K + bb * C::OP_TILE + row_off;
+      uint8_t* sv = smem + C::OFF_V + bb * C::OP_TILE + row_off;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const int j = ((c >> 1) + rot) & 7;  // 16-byte raw chunk (c>>1) rotated
         const int chunk8 = 2 * j + (c & 1);  // which 8 head-dim elements
-        *reinterpret_cast<uint4*>(sk + chunk8 * 128) = e4m3x8_to_f16x8(kr[c]);
+        const int off = (chunk8 >> 3) * C::KV_HALF + (((chunk8 & 7) ^ (t & 7)) << 4);
+        *reinterpret_cast<uint4*>(sk + off) = e4m3x8_to_f16x8(kr[c]);
         const uint4 vv = v_zero ? make_uint4(0, 0, 0, 0) : e4m3x8_to_f16x8(vr[c]);
-        *reinterpret_cast<uint4*>(sv + chunk8 * 128) = vv;
+        *reinterpret_cast<uint4*>(sv + off) = vv;
       }
       fence_proxy_async_smem();
       mbar_arrive(&kv_ready[bb]);
@@ -426,53 +463,66 @@ __global__ void __launch_bounds__(TcCfg<NT>::THREADS, 1) split_tc_kernel(const S
       constexpr uint32_t idesc_s = umma_idesc_f16(128, NT, false, false);  // K, Q both K-major
       constexpr uint32_t idesc_o = umma_idesc_f16(128, NT, true, true);    // V^T, P^T MN-major
       const uint32_t sbase = smem_addr(smem);
-      auto issue_s = [&](int n) {
+      auto issue_s = [&](int n) {  // S^T = K Q^T, K = head_dim in steps of 16
         const int bb = n & 1;
         const uint32_t ka = sbase + C::OFF_K + bb * C::OP_TILE;
         const uint32_t qa = sbase + C::OFF_Q;
 #pragma unroll
         for (int s = 0; s < C::D / 16; ++s)
-          umma_f16(tmem + C::COL_S + bb * NT, umma_desc(ka + s * 256, 128, 2048),
-                   umma_desc(qa + s * 256, 128, 2048), idesc_s, s > 0);
+          umma_f16(tmem + C::COL_S + bb * NT,
+                   umma_desc(ka + (s >> 2) * C::KV_HALF + (s & 3) * 32, 16, 1024, kSw128),
+                   umma_desc(qa + (s >> 2) * C::Q_HALF + (s & 3) * 32, 16, 1024, kSw128),
+                   idesc_s, s > 0);
         umma_commit(&s_full[bb]);
       };
-      auto issue_o = [&](int n) {
+      auto issue_o = [&](int n) {  // O^T = V^T P^T, K = tokens in steps of 16
         const int bb = n & 1;
         const uint32_t va = sbase + C::OFF_V + bb * C::OP_TILE;
         const uint32_t pa = sbase + C::OFF_P + bb * C::P_BYTES;
 #pragma unroll
         for (int s = 0; s < C::TILE / 16; ++s)
-          umma_f16(tmem + C::COL_O + bb * NT, umma_desc(va + s * 4096, 2048, 128),
-                   umma_desc(pa + s * 2 * C::P_LBO, C::P_LBO, 128), idesc_o, s > 0);
+          umma_f16(tmem + C::COL_O + bb * NT, umma_desc(va + s * 2048, C::KV_HALF, 1024, kSw128),
+                   umma_desc(pa + s * 2 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE), idesc_o,
+                   s > 0);
         umma_commit(&o_full[bb]);
       };
-      bool ok = true;
+      // Event-driven issue: S^T of tile k once its K tile is converted and
+      // softmax(k-2) has read S^T buffer k&1; O^T of tile k once softmax(k)
+      // has written P^T and O^T buffer k&1 has been read back (tile k-2).
       int s_issued = 0, o_issued = 0;
-      if (ntiles > 0) {
-        ok = mbar_wait(&kv_ready[0], 0, a.err);
-        if (ok) {
-          tmem_fence_after();
-          issue_s(0);
-          s_issued = 1;
+      bool ok = true;
+      const long long start = clock64();
+      long long last = start;
+      while (o_issued < ntiles) {
+        bool progress = false;
+        if (s_issued < ntiles && s_issued < o_issued + 2) {
+          const int k = s_issued;
+          if (mbar_test(&kv_ready[k & 1], (k >> 1) & 1) &&
+              (k < 2 || mbar_test(&p_ready[k & 1], ((k - 2) >> 1) & 1))) {
+            tmem_fence_after();
+            issue_s(k);
+            ++s_issued;
+            progress = true;
+          }
         }
-      }
-      for (int n = 0; ok && n < ntiles; ++n) {
-        if (*abort_flag) break;
-        if (n + 1 < ntiles) {  // S^T of the next tile while softmax works on this one
-          const int nb = (n + 1) & 1;
-          ok = mbar_wait(&kv_ready[nb], ((n + 1) >> 1) & 1, a.err);
-          if (ok && n >= 1) ok = mbar_wait(&p_ready[nb], ((n - 1) >> 1) & 1, a.err);
-          if (!ok) break;
-          tmem_fence_after();
-          issue_s(n + 1);
-          s_issued = n + 2;
+        if (o_issued < s_issued) {
+          const int k = o_issued;
+          if (mbar_test(&p_ready[k & 1], (k >> 1) & 1) &&
+              (k < 2 || mbar_test(&o_free[k & 1], ((k - 2) >> 1) & 1))) {
+            tmem_fence_after();
+            issue_o(k);
+            ++o_issued;
+            progress = true;
+          }
         }
-        ok = mbar_wait(&p_ready[n & 1], (n >> 1) & 1, a.err);
-        if (ok && n >= 2) ok = mbar_wait(&o_free[n & 1], ((n - 2) >> 1) & 1, a.err);
-        if (!ok) break;
-        tmem_fence_after();
-        issue_o(n);
-        o_issued = n + 1;
+        const long long now = clock64();
+        if (progress) {
+          last = now;
+        } else if (now - last > kWaitTimeoutCycles || *abort_flag) {
+          if (!*abort_flag) record_error_at(a.err, kErrTimeout);
+          ok = false;
+          break;
+        }
       }
       if (!ok) *abort_flag = 1;
       if (*abort_flag) {
@@ -594,7 +644,11 @@ __global__ void __launch_bounds__(TcCfg<NT>::THREADS, 1) split_tc_kernel(const S
           l_part[r] = fmaf(l_part[r], av[e], p[r]);
         }
       }
-      uint8_t* sp = smem + C::OFF_P + bb * C::P_BYTES + (i >> 3) * C::P_LBO + (i & 7) * 16;
+      // token i's row of P^T: NT f16 = NT/8 chunks of 16 B, XOR-swizzled by
+      // the row's position in its 8-token atom (SW64: bits 7-8 of the
+      // address, i.e. row >> 1; SW32: bit 7, i.e. row >> 2)
+      uint8_t* sp = smem + C::OFF_P + bb * C::P_BYTES + (i >> 3) * C::P_SBO + (i & 7) * C::P_ROW;
+      const int pswz = NT == 32 ? ((i & 7) >> 1) & 3 : ((i & 7) >> 2) & 1;
 #pragma unroll
       for (int g = 0; g < NT / 8; ++g) {
         uint4 w;
@@ -602,7 +656,7 @@ __global__ void __launch_bounds__(TcCfg<NT>::THREADS, 1) split_tc_kernel(const S
         w.y = pack_f16x2(p[8 * g + 2], p[8 * g + 3]);
         w.z = pack_f16x2(p[8 * g + 4], p[8 * g + 5]);
         w.w = pack_f16x2(p[8 * g + 6], p[8 * g + 7]);
-        *reinterpret_cast<uint4*>(sp + g * 128) = w;
+        *reinterpret_cast<uint4*>(sp + ((g ^ pswz) << 4)) = w;
       }
       fence_proxy_async_smem();
       tmem_fence_before();
