@@ -17,6 +17,7 @@ ranks. Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -160,6 +161,25 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    record (profiles/dram_traffic.json), or None when there is no record for
+    the workload or the kernel sources changed since the counters were
+    taken (the record stores their sha256)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f)[workload_name]
+        h = hashlib.sha256()
+        for src in rec["source_files"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        return rec.get("dram_bytes_per_launch_full")
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def algorithmic_bytes(wl: W.Workload, kv_lens):
@@ -395,7 +415,9 @@ def run_ours(args, rank, world, local):
         },
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": None,
+            "frac": achieved / peak,
+            "traffic": None if args.batch else recorded_traffic(wl.name),
+            "traffic_unit": "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)",
             "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
             "frac_of_8tbs_spec": achieved / 8000.0,
             "kernel": "split_fma_kernel" + (" + merge_states_kernel" if splits > 1 else ""),
