@@ -46,6 +46,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0: planner)")
+    ap.add_argument("--tensor-cores", action="store_true",
+                    help="bf16 K/V: use the tensor-core kernel instead of the FMA kernel")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (profiling a smaller case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -287,15 +289,16 @@ def run_ours(args, rank, world, local):
     max_len = int(kl.max().item())
     out = torch.empty((wl.batch, wl.q_len, wl.num_q_heads, wl.head_dim), dtype=torch.float32, device=dev)
     lse = torch.empty((wl.batch, wl.q_len, wl.num_q_heads), dtype=torch.float32, device=dev)
+    flags = B.PDA_FLAG_TENSOR_CORES if args.tensor_cores else 0
     kw = dict(num_kv_heads=wl.num_kv_heads, scale=scale, causal_offset=wl.causal_offset,
               window=wl.window, kv_scale=inp["kv_scale"], max_kv_len=max_len,
-              num_splits=args.splits)
+              num_splits=args.splits, flags=flags)
     params = B.make_params(
         batch=wl.batch, q_len=wl.q_len, num_q_heads=wl.num_q_heads,
         num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, page_size=wl.page_size,
         max_pages_per_seq=pt.shape[1], num_pages=kp.shape[0], scale=scale,
         causal_offset=wl.causal_offset, window=wl.window, kv_dtype=wl.kv_dtype,
-        kv_scale=inp["kv_scale"], max_kv_len=max_len, num_splits=args.splits)
+        kv_scale=inp["kv_scale"], max_kv_len=max_len, num_splits=args.splits, flags=flags)
     ws_bytes = B.workspace_bytes(params)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()

@@ -78,6 +78,8 @@ typedef enum {
 
 /* flags */
 #define PDA_FLAG_NO_PDL 1u  /* launch the merge without programmatic dependent launch */
+#define PDA_FLAG_TENSOR_CORES 2u /* bf16 K/V, head_dim 128: use the tensor-core kernel
+                                    (FP8 K/V with > 8 packed rows always does) */
 
 typedef struct {
   int32_t batch;            /* B >= 0 */

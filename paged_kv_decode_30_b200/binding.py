@@ -20,6 +20,7 @@ PDA_KV_FP8_E4M3 = 1
 PDA_CAUSAL_OFF = -1
 PDA_CAUSAL_BOTTOM_RIGHT = -2
 PDA_FLAG_NO_PDL = 1
+PDA_FLAG_TENSOR_CORES = 2
 # Size of the library's fixed partials array used by paged_decode_attn_no_alloc.
 PDA_NO_ALLOC_WORKSPACE_BYTES = 16 * 1024 * 1024
 

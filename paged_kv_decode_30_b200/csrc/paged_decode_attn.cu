@@ -17,6 +17,7 @@
 #include "merge.cuh"
 #include "paged_decode_attn.h"
 #include "split_tc.cuh"
+#include "split_tma.cuh"
 #include "split_variants.cuh"
 
 namespace pda {
@@ -79,11 +80,18 @@ struct Plan {
   bool tc;                 // tensor-core kernel (else the FMA kernel)
 };
 
+// TMA coordinates are 32-bit: the pool's rows must fit.
+bool pool_rows_fit(const pda_params* p) {
+  return (long long)p->num_pages * p->num_kv_heads * p->page_size < (1ll << 31);
+}
+
 // The tensor-core kernel takes FP8 K/V with head_dim 128 when the packed
 // rows of a kv head (G * q_len) exceed what the FMA kernel holds in one CTA
 // (8): then QK^T and PV are real dense contractions (N = 16 or 32 rows).
 bool use_tensor_cores(const pda_params* p, int M) {
-  return p->kv_dtype == PDA_KV_FP8_E4M3 && p->head_dim == 128 && M > 8 && p->page_size >= 8;
+  if (p->head_dim != 128 || p->page_size < 8 || !pool_rows_fit(p)) return false;
+  if (p->kv_dtype == PDA_KV_FP8_E4M3) return M > 8;
+  return (p->flags & PDA_FLAG_TENSOR_CORES) != 0;  // bf16: opt-in
 }
 
 pda_status validate(const pda_params* p) {
@@ -116,7 +124,10 @@ Plan make_plan(const pda_params* p) {
   pl.rows = (long long)p->batch * p->q_len * p->num_q_heads;
   pl.tc = use_tensor_cores(p, pl.M);
   if (pl.tc) {
-    pl.mt = pl.M <= 16 ? 16 : 32;  // rows per CTA (MMA N)
+    if (p->kv_dtype == PDA_KV_FP8_E4M3)
+      pl.mt = pl.M <= 16 ? 16 : 32;  // rows per CTA; MMA N = 2 * rows for S^T
+    else
+      pl.mt = pl.M <= 4 ? 4 : 8;     // bf16: N = 16 holds P^T hi and lo rows
     pl.tw = 128;                   // tokens per tile (MMA M)
     pl.tiles_per_cta_iter = 128;
   } else {
@@ -310,7 +321,7 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   cudaError_t e;
   const int kv = fp8 ? 1 : 0;
   if (pl.tc) {
-    e = launch_split_tc(pl.mt, a, grid, stream);
+    e = launch_split_tma(kv, pl.mt, k_pages, v_pages, a, grid, stream);
   } else switch (p.head_dim) {
     case 64: e = launch_split_d64(kv, pl.mt, pl.tw, a, grid, stream); break;
     case 128: e = launch_split_d128(kv, pl.mt, pl.tw, a, grid, stream); break;

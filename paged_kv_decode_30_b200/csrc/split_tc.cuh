@@ -230,6 +230,22 @@ __device__ __forceinline__ bool named_bar_and(int id, int threads, bool v) {
   return r != 0;
 }
 
+// One named barrier returning the OR of `want` over the threads; `*ok_out`
+// gets the AND of `ok`. (Two barrier reductions back to back on the same id.)
+__device__ __forceinline__ bool named_bar_or_and(int id, int threads, bool want, bool ok,
+                                                 bool* ok_out) {
+  uint32_t r_or, r_and;
+  asm volatile(
+      "{\n\t.reg .pred p, q, x, y;\n\tsetp.ne.u32 p, %2, 0;\n\tsetp.ne.u32 q, %3, 0;\n\t"
+      "bar.red.or.pred x, %4, %5, p;\n\tbar.red.and.pred y, %4, %5, q;\n\t"
+      "selp.u32 %0, 1, 0, x;\n\tselp.u32 %1, 1, 0, y;\n\t}"
+      : "=r"(r_or), "=r"(r_and)
+      : "r"((uint32_t)want), "r"((uint32_t)ok), "r"(id), "r"(threads)
+      : "memory");
+  *ok_out = r_and != 0;
+  return r_or != 0;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
                : "memory");

@@ -89,6 +89,19 @@ def test_parity_vs_oracle(lib, case, splits):
     U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, f"{case.name}/s={splits}")
 
 
+TC_BF16_CASES = [c for c in CASES if c.kv_dtype == BF16 and c.head_dim == 128]
+
+
+@pytest.mark.parametrize("case", TC_BF16_CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("splits", [0, 1, 3, 64])
+def test_parity_tensor_core_bf16(lib, case, splits):
+    """bf16 K/V through the tensor-core kernel (opt-in flag)."""
+    inp = W.generate(case)
+    ref_out, ref_lse = U.run_oracle(inp)
+    out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=B.PDA_FLAG_TENSOR_CORES)
+    U.assert_parity(out, lse, ref_out, ref_lse, BF16, f"{case.name}/tc/s={splits}")
+
+
 @pytest.mark.parametrize("case", [CASES[2], CASES[5], CASES[7]], ids=lambda w: w.name)
 def test_page_permutation_invariance(lib, case):
     inp = W.generate(case)
@@ -193,6 +206,15 @@ def test_full_size_sampled(lib, name, seqs):
     ref_out, ref_lse = U.run_oracle(inp, seqs=seqs)
     U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, case.kv_dtype, name)
     assert np.isfinite(out).all()
+
+
+def test_full_size_headline_tensor_core_bf16(lib):
+    case = W.HEADLINE
+    inp = W.generate(case, device="cuda")
+    out, lse, _ = U.run_cuda(inp, flags=B.PDA_FLAG_TENSOR_CORES)
+    seqs = [3, 64, 126]
+    ref_out, ref_lse = U.run_oracle(inp, seqs=seqs)
+    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, BF16, "headline/tc")
 
 
 @pytest.mark.parametrize("name", [W.VARLEN.name, W.LONGCTX.name])
