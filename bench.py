@@ -36,6 +36,7 @@ from paged_kv_decode_30_b200 import workloads as W  # noqa: E402
 
 METRIC = "paged decode attn: tokens/s and achieved HBM GB/s (% of B200 roofline), 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126e6  # B200 L2
 
 
 def parse_args(argv=None):
@@ -46,13 +47,15 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0: planner)")
-    ap.add_argument("--tensor-cores", action="store_true",
-                    help="bf16 K/V: use the tensor-core kernel instead of the FMA kernel")
+    ap.add_argument("--kernel", choices=["auto", "tensor_cores", "cuda_cores"], default="auto",
+                    help="split kernel: the planner's choice, or force one")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (profiling a smaller case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the read-only HBM probe and the CUDA-graph replay (profiling runs)")
     return ap.parse_args(argv)
 
 
@@ -165,14 +168,15 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def recorded_traffic(workload_name: str):
+def recorded_traffic(workload_name: str, kernel_name: str):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    record (profiles/dram_traffic.json), or None when there is no record for
-    the workload or the kernel sources changed since the counters were
-    taken (the record stores their sha256)."""
+    record (profiles/dram_traffic.json, keyed "<workload>/<kernel>"), or None
+    when there is no record for that workload and kernel or the kernel
+    sources changed since the counters were taken (the record stores their
+    sha256)."""
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
-            rec = json.load(f)[workload_name]
+            rec = json.load(f)[f"{workload_name}/{kernel_name}"]
         h = hashlib.sha256()
         for src in rec["source_files"]:
             with open(os.path.join(ROOT, src), "rb") as f:
@@ -222,19 +226,63 @@ def oracle_units(inp, units):
     return elapsed
 
 
+def oracle_sequences_mt(inp, first: int, count: int, threads: int) -> float:
+    """Whole sequences [first, first + count), all heads, on `threads`
+    OpenMP threads of the oracle (one row per task). Returns seconds."""
+    from oracle import oracle as orc
+    wl = inp["workload"]
+    sl = slice(first, first + count)
+    args = (W.to_bits(inp["q"][sl].contiguous()), W.to_bits(inp["k_pages"]),
+            W.to_bits(inp["v_pages"]), inp["page_table"][sl].contiguous().cpu().numpy(),
+            inp["kv_lens"][sl].contiguous().cpu().numpy())
+    t0 = time.perf_counter()
+    orc.paged_decode_attn(*args, num_kv_heads=wl.num_kv_heads, page_size=wl.page_size,
+                          scale=W.scale_of(wl), causal_offset=wl.causal_offset,
+                          window=wl.window, kv_dtype=wl.kv_dtype,
+                          kv_scale=inp["kv_scale"], threads=threads)
+    return time.perf_counter() - t0
+
+
+def host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def cpu_baseline(inp, seconds: float):
+    """The oracle timed on the host: single-threaded on (sequence, kv head)
+    units, then on every host core (OpenMP) on whole sequences, each leg on
+    a bounded sample of about `seconds`. The reported value is the
+    all-cores leg; the single-threaded one rides along."""
     wl = inp["workload"]
     units, elapsed = 0, 0.0
     order = [(b, g) for b in range(wl.batch) for g in range(wl.num_kv_heads)]
     while elapsed < seconds and units < len(order):
         elapsed += oracle_units(inp, [order[units]])
         units += 1
-    tokens = units / wl.num_kv_heads * wl.q_len
-    return {
-        "value": tokens / elapsed, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+    single = {
+        "value": units / wl.num_kv_heads * wl.q_len / elapsed, "unit": "tokens/s", "cores": 1,
         "sample": (f"{units} (sequence, kv head) units of {wl.name} "
                    f"({units / wl.num_kv_heads:.3f} full sequences, all heads), "
                    f"single-threaded fp64 C oracle, {elapsed:.1f} s"),
+    }
+    threads = host_threads()
+    seqs, mt_elapsed = 0, 0.0
+    # the K/V pools go to the host once; each call then takes whole sequences
+    host = dict(inp, q=inp["q"].cpu(), k_pages=inp["k_pages"].cpu(),
+                v_pages=inp["v_pages"].cpu(), page_table=inp["page_table"].cpu(),
+                kv_lens=inp["kv_lens"].cpu())
+    while mt_elapsed < seconds and seqs < wl.batch:
+        n = min(max(1, threads // max(1, wl.num_q_heads * wl.q_len) + 1), wl.batch - seqs)
+        mt_elapsed += oracle_sequences_mt(host, seqs, n, threads)
+        seqs += n
+    return {
+        "value": seqs * wl.q_len / mt_elapsed, "unit": "tokens/s", "cores": threads,
+        "kind": "oracle",
+        "sample": (f"{seqs} full sequences (all heads) of {wl.name}, fp64 C oracle on "
+                   f"{threads} OpenMP threads (one output row per task), {mt_elapsed:.1f} s"),
+        "single_thread": single,
     }
 
 
@@ -289,7 +337,8 @@ def run_ours(args, rank, world, local):
     max_len = int(kl.max().item())
     out = torch.empty((wl.batch, wl.q_len, wl.num_q_heads, wl.head_dim), dtype=torch.float32, device=dev)
     lse = torch.empty((wl.batch, wl.q_len, wl.num_q_heads), dtype=torch.float32, device=dev)
-    flags = B.PDA_FLAG_TENSOR_CORES if args.tensor_cores else 0
+    flags = {"auto": 0, "tensor_cores": B.PDA_FLAG_TENSOR_CORES,
+             "cuda_cores": B.PDA_FLAG_CUDA_CORES}[args.kernel]
     kw = dict(num_kv_heads=wl.num_kv_heads, scale=scale, causal_offset=wl.causal_offset,
               window=wl.window, kv_scale=inp["kv_scale"], max_kv_len=max_len,
               num_splits=args.splits, flags=flags)
@@ -299,12 +348,21 @@ def run_ours(args, rank, world, local):
         max_pages_per_seq=pt.shape[1], num_pages=kp.shape[0], scale=scale,
         causal_offset=wl.causal_offset, window=wl.window, kv_dtype=wl.kv_dtype,
         kv_scale=inp["kv_scale"], max_kv_len=max_len, num_splits=args.splits, flags=flags)
+    kernel_name = B.KERNEL_NAMES.get(B.plan_kernel(params), "unknown")
     ws_bytes = B.workspace_bytes(params)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
         return B.paged_decode_attn(q, kp, vp, pt, kl, out=out, lse=lse, workspace=ws, **kw)[2]
+
+    # K/V smaller than twice the L2 (126 MB) could stay cached between
+    # steps: then every timed step is preceded by a 256 MiB write (outside
+    # the step's events) and the value comes from the per-step events.
+    _, kv_bytes0 = algorithmic_bytes(wl, kl.tolist())
+    flush = None
+    if kv_bytes0 < 2 * L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     splits = step()
     torch.cuda.synchronize()
@@ -324,6 +382,8 @@ def run_ours(args, rank, world, local):
     t_end = torch.cuda.Event(enable_timing=True)
     t_begin.record(stream)
     for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
         starts[i].record(stream)
         step()
         ends[i].record(stream)
@@ -333,6 +393,8 @@ def run_ours(args, rank, world, local):
     clocks = sampler.stop()
     elapsed_ms = t_begin.elapsed_time(t_end)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if flush is not None:  # the flushes are not part of the job
+        elapsed_ms = sum(step_ms)
     if B.last_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
 
@@ -344,6 +406,53 @@ def run_ours(args, rank, world, local):
     achieved = alg_bytes / (avg_launch_ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     launches_per_step = 1 + (1 if splits > 1 else 0)
+
+    # Read-only HBM probe in the same run (our streaming-load kernel over a
+    # 4 GiB buffer, larger than L2): the ceiling for a kernel that only reads.
+    probe_gbs = None
+    try:
+        if args.no_extras:
+            raise RuntimeError("skipped (--no-extras)")
+        pbuf = torch.zeros(4 * 1024 ** 3, dtype=torch.uint8, device=dev)
+        sink = torch.zeros(1, dtype=torch.int64, device=dev)
+        for _ in range(3):
+            B.hbm_read_probe(pbuf, sink)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        p0.record(stream)
+        for _ in range(reps):
+            B.hbm_read_probe(pbuf, sink)
+        p1.record(stream)
+        torch.cuda.synchronize()
+        probe_gbs = pbuf.numel() * reps / (p0.elapsed_time(p1) / 1e3) / 1e9
+        del pbuf
+    except (RuntimeError, B.PdaError) as e:  # out of memory: report none
+        print(f"read probe skipped: {e}", file=sys.stderr)
+
+    # One call captured in a CUDA graph and replayed (no host launch gaps;
+    # L2 not flushed between replays).
+    graph = None
+    try:
+        if args.no_extras:
+            raise RuntimeError("skipped (--no-extras)")
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        n_g = max(20, min(args.steps, 500))
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(n_g):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        g_ms = g0.elapsed_time(g1) / n_g
+        graph = {"ms_per_step": g_ms, "value": tokens_per_step * world / (g_ms / 1e3),
+                 "unit": "tokens/s", "replays": n_g, "l2": "warm (no flush between replays)"}
+        del g
+    except RuntimeError as e:
+        graph = {"error": str(e).splitlines()[0][:200]}
 
     # End to end through the public API with host buffers: every step copies
     # the step's inputs (q, page table, kv lengths) from pinned host memory
@@ -411,23 +520,27 @@ def run_ours(args, rank, world, local):
             "kv_len": max_len if wl.kv_lens[0] == "const" else str(wl.kv_lens),
             "causal_offset": wl.causal_offset, "window": wl.window,
             "num_splits": splits, "parallelism": f"replicas x{world}",
-            "l2": "no flush: K/V read per step "
-                  f"({kv_bytes / 1e9:.2f} GB) larger than L2" if kv_bytes > 126e6
-                  else "inputs smaller than L2",
+            "l2": ("flushed before every timed step (256 MiB write, outside the step's "
+                   "events; value from the per-step events)") if flush is not None
+                  else f"no flush: K/V read per step ({kv_bytes / 1e9:.2f} GB) is more than "
+                       "twice the L2",
             "algorithmic_bytes_per_step": alg_bytes,
         },
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": None if args.batch else recorded_traffic(wl.name),
+            "traffic": None if args.batch else recorded_traffic(wl.name, kernel_name),
             "traffic_unit": "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)",
             "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
             "frac_of_8tbs_spec": achieved / 8000.0,
-            "kernel": "split_fma_kernel" + (" + merge_states_kernel" if splits > 1 else ""),
+            "kernel": kernel_name + (" + merge_states_kernel" if splits > 1 else ""),
+            "read_probe_gbs": probe_gbs,
+            "frac_of_read_probe": achieved / probe_gbs if probe_gbs else None,
             "avg_launch_ms": avg_launch_ms,
         },
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "graph": graph,
         "e2e": e2e,
         "cpu_baseline": cpu,
     }

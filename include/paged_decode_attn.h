@@ -78,8 +78,9 @@ typedef enum {
 
 /* flags */
 #define PDA_FLAG_NO_PDL 1u  /* launch the merge without programmatic dependent launch */
-#define PDA_FLAG_TENSOR_CORES 2u /* bf16 K/V, head_dim 128: use the tensor-core kernel
-                                    (FP8 K/V with > 8 packed rows always does) */
+#define PDA_FLAG_TENSOR_CORES 2u /* use the tensor-core kernel wherever it applies
+                                    (head_dim 128), not only where the planner picks it */
+#define PDA_FLAG_CUDA_CORES 4u   /* always use the CUDA-core (FMA) kernel */
 
 typedef struct {
   int32_t batch;            /* B >= 0 */
@@ -206,6 +207,32 @@ PDA_API int32_t pda_choose_num_splits(const pda_params* params, int32_t num_sms)
 PDA_API pda_status pda_merge_states(const float* o_parts, const float* lse_parts,
                             int32_t num_splits, int64_t rows, int32_t head_dim,
                             float* out, float* lse, pda_stream_t stream);
+
+/* Which split kernel paged_decode_attn would launch for these params
+ * (host-only; the planner's choice):
+ *   PDA_KERNEL_SPLIT_TMA  tensor-core kernel (2D TMA tiles of 128 tokens,
+ *                         tcgen05 MMAs with TMEM accumulators): head_dim 128
+ *                         with bf16 K/V and at most 8 packed rows per kv head
+ *                         (G * q_len), or FP8 K/V and more than 8; any
+ *                         head_dim-128 case with PDA_FLAG_TENSOR_CORES;
+ *   PDA_KERNEL_SPLIT_FMA  CUDA-core kernel (warp-shuffle FMAs, cp.async.bulk
+ *                         page copies): everything else, and every case with
+ *                         PDA_FLAG_CUDA_CORES.
+ * Returns -1 if the params are invalid. */
+#define PDA_KERNEL_SPLIT_FMA 0
+#define PDA_KERNEL_SPLIT_TMA 1
+PDA_API int32_t pda_plan_kernel(const pda_params* params);
+
+/*
+ * Measurement helper, not part of the attention path: reads `bytes` bytes at
+ * `buf` once with 128-bit streaming loads (4 CTAs of 512 threads per SM) and
+ * XORs the words into *sink, so a caller can time the device's read-only
+ * HBM bandwidth with the same events and in the same run as the attention
+ * call. buf and bytes 16-byte aligned, sink 8-byte aligned device memory
+ * (its value is meaningless). Asynchronous on `stream`.
+ */
+PDA_API pda_status pda_hbm_read_probe(const void* buf, size_t bytes, uint64_t* sink,
+                                      pda_stream_t stream);
 
 /* Human-readable name of a status. Never NULL. */
 PDA_API const char* pda_status_string(pda_status status);

@@ -40,7 +40,7 @@
  * e4m3/bf16 decode against torch's independent float8/bfloat16 casts, and
  * hand-derived golden fixtures.
  *
- * Build: gcc -O2 -ffp-contract=off -fPIC -shared oracle.c -o liboracle.so -lm
+ * Build: gcc -O2 -ffp-contract=off -fopenmp -fPIC -shared oracle.c -o liboracle.so -lm
  */
 #include <math.h>
 #include <stdint.h>
@@ -110,6 +110,97 @@ static int key_visible(int64_t j, int64_t kv_len, int causal, int64_t pos,
   return 1;
 }
 
+/* Shared argument checks of the two entry points below. */
+static int check_args(const int32_t* kv_lens, int B, int q_len, int Hq, int Hkv,
+                      int D, int page_size, int max_pages, int num_pages,
+                      int causal_offset, int kv_dtype, int64_t* max_len) {
+  if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || D < 1 || page_size < 1 ||
+      max_pages < 0 || num_pages < 0 || Hq % Hkv != 0)
+    return ORACLE_BAD_ARG;
+  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3)
+    return ORACLE_BAD_ARG;
+  if (causal_offset < ORACLE_CAUSAL_BOTTOM_RIGHT) return ORACLE_BAD_ARG;
+  *max_len = 0;
+  for (int b = 0; b < B; ++b) {
+    if (kv_lens[b] < 0) return ORACLE_BAD_ARG;
+    if (kv_lens[b] > (int64_t)max_pages * page_size) return ORACLE_BAD_ARG;
+    if (kv_lens[b] > *max_len) *max_len = kv_lens[b];
+  }
+  return ORACLE_OK;
+}
+
+/*
+ * One output row: out[b, i, h, :] and lse[b, i, h], restricted to keys in
+ * [tok_lo, tok_hi) (tok_hi < 0 means no restriction). `s` is scratch for
+ * kv_lens[b] scores.
+ */
+static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_pages,
+                      const int32_t* page_table, const int32_t* kv_lens, int q_len,
+                      int Hq, int Hkv, int D, int page_size, int max_pages,
+                      int num_pages, float scale, int causal_offset, int window,
+                      int kv_dtype, float kv_scale, int64_t tok_lo, int64_t tok_hi,
+                      int b, int i, int h, double* s, double* out, double* lse) {
+  const int G = Hq / Hkv;
+  const int causal = causal_offset != ORACLE_CAUSAL_OFF;
+  const double dscale = (double)scale;
+  const double dkv_scale = (double)kv_scale;
+  const int64_t L = kv_lens[b];
+  const int64_t pos = row_position(causal_offset, L, q_len, i);
+  const int g = h / G; /* reading R4 */
+  const uint16_t* qrow = q + (((int64_t)b * q_len + i) * Hq + h) * D;
+  double* orow = out + (((int64_t)b * q_len + i) * Hq + h) * D;
+  double* lrow = lse + ((int64_t)b * q_len + i) * Hq + h;
+
+  /* Pass 1: scores of the visible keys, walking the page table. */
+  double m = -INFINITY;
+  int64_t nvis = 0;
+  for (int64_t j = 0; j < L; ++j) {
+    int vis = key_visible(j, L, causal, pos, window);
+    if (vis && tok_hi >= 0 && (j < tok_lo || j >= tok_hi)) vis = 0;
+    if (!vis) {
+      s[j] = -INFINITY;
+      continue;
+    }
+    const int32_t page = page_table[(int64_t)b * max_pages + j / page_size];
+    if (page < 0 || page >= num_pages) return ORACLE_BAD_PAGE;
+    const int64_t row = j % page_size;
+    const int64_t base = (((int64_t)page * Hkv + g) * page_size + row) * D;
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d)
+      dot += oracle_bf16_to_double(qrow[d]) *
+             kv_elem(k_pages, kv_dtype, dkv_scale, base + d);
+    s[j] = dscale * dot;
+    if (s[j] > m) m = s[j];
+    ++nvis;
+  }
+
+  if (nvis == 0) { /* reading R8 */
+    for (int d = 0; d < D; ++d) orow[d] = 0.0;
+    *lrow = -INFINITY;
+    return ORACLE_OK;
+  }
+
+  /* lse = m + ln sum_j exp(s_j - m)  (reading R1) */
+  double sum = 0.0;
+  for (int64_t j = 0; j < L; ++j)
+    if (s[j] != -INFINITY) sum += exp(s[j] - m);
+  const double row_lse = m + log(sum);
+  *lrow = row_lse;
+
+  /* Pass 2: out = sum_j exp(s_j - lse) * v_j. */
+  for (int d = 0; d < D; ++d) orow[d] = 0.0;
+  for (int64_t j = 0; j < L; ++j) {
+    if (s[j] == -INFINITY) continue;
+    const double p = exp(s[j] - row_lse);
+    const int32_t page = page_table[(int64_t)b * max_pages + j / page_size];
+    const int64_t row = j % page_size;
+    const int64_t base = (((int64_t)page * Hkv + g) * page_size + row) * D;
+    for (int d = 0; d < D; ++d)
+      orow[d] += p * kv_elem(v_pages, kv_dtype, dkv_scale, base + d);
+  }
+  return ORACLE_OK;
+}
+
 /*
  * out[b, i, h, :] and lse[b, i, h] for every row, restricted to keys in
  * [tok_lo, tok_hi) (tok_hi < 0 means no restriction). The restriction lets
@@ -128,92 +219,76 @@ int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
                              int window, int kv_dtype, float kv_scale,
                              int64_t tok_lo, int64_t tok_hi, double* out,
                              double* lse) {
-  if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || D < 1 || page_size < 1 ||
-      max_pages < 0 || num_pages < 0 || Hq % Hkv != 0)
-    return ORACLE_BAD_ARG;
-  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3)
-    return ORACLE_BAD_ARG;
-  if (causal_offset < ORACLE_CAUSAL_BOTTOM_RIGHT) return ORACLE_BAD_ARG;
-
-  const int G = Hq / Hkv;
-  const int causal = causal_offset != ORACLE_CAUSAL_OFF;
-  const double dscale = (double)scale;
-  const double dkv_scale = (double)kv_scale;
-
-  int64_t max_len = 0;
-  for (int b = 0; b < B; ++b) {
-    if (kv_lens[b] < 0) return ORACLE_BAD_ARG;
-    if (kv_lens[b] > (int64_t)max_pages * page_size) return ORACLE_BAD_ARG;
-    if (kv_lens[b] > max_len) max_len = kv_lens[b];
-  }
+  int64_t max_len;
+  int st = check_args(kv_lens, B, q_len, Hq, Hkv, D, page_size, max_pages, num_pages,
+                      causal_offset, kv_dtype, &max_len);
+  if (st != ORACLE_OK) return st;
   double* s = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
   if (!s) return ORACLE_NO_MEMORY;
-
-  for (int b = 0; b < B; ++b) {
-    const int64_t L = kv_lens[b];
-    for (int i = 0; i < q_len; ++i) {
-      const int64_t pos = row_position(causal_offset, L, q_len, i);
+  for (int b = 0; b < B; ++b)
+    for (int i = 0; i < q_len; ++i)
       for (int h = 0; h < Hq; ++h) {
-        const int g = h / G; /* reading R4 */
-        const uint16_t* qrow = q + (((int64_t)b * q_len + i) * Hq + h) * D;
-        double* orow = out + (((int64_t)b * q_len + i) * Hq + h) * D;
-        double* lrow = lse + ((int64_t)b * q_len + i) * Hq + h;
-
-        /* Pass 1: scores of the visible keys, walking the page table. */
-        double m = -INFINITY;
-        int64_t nvis = 0;
-        for (int64_t j = 0; j < L; ++j) {
-          int vis = key_visible(j, L, causal, pos, window);
-          if (vis && tok_hi >= 0 && (j < tok_lo || j >= tok_hi)) vis = 0;
-          if (!vis) {
-            s[j] = -INFINITY;
-            continue;
-          }
-          const int32_t page = page_table[(int64_t)b * max_pages + j / page_size];
-          if (page < 0 || page >= num_pages) {
-            free(s);
-            return ORACLE_BAD_PAGE;
-          }
-          const int64_t row = j % page_size;
-          const int64_t base = (((int64_t)page * Hkv + g) * page_size + row) * D;
-          double dot = 0.0;
-          for (int d = 0; d < D; ++d)
-            dot += oracle_bf16_to_double(qrow[d]) *
-                   kv_elem(k_pages, kv_dtype, dkv_scale, base + d);
-          s[j] = dscale * dot;
-          if (s[j] > m) m = s[j];
-          ++nvis;
-        }
-
-        if (nvis == 0) { /* reading R8 */
-          for (int d = 0; d < D; ++d) orow[d] = 0.0;
-          *lrow = -INFINITY;
-          continue;
-        }
-
-        /* lse = m + ln sum_j exp(s_j - m)  (reading R1) */
-        double sum = 0.0;
-        for (int64_t j = 0; j < L; ++j)
-          if (s[j] != -INFINITY) sum += exp(s[j] - m);
-        const double row_lse = m + log(sum);
-        *lrow = row_lse;
-
-        /* Pass 2: out = sum_j exp(s_j - lse) * v_j. */
-        for (int d = 0; d < D; ++d) orow[d] = 0.0;
-        for (int64_t j = 0; j < L; ++j) {
-          if (s[j] == -INFINITY) continue;
-          const double p = exp(s[j] - row_lse);
-          const int32_t page = page_table[(int64_t)b * max_pages + j / page_size];
-          const int64_t row = j % page_size;
-          const int64_t base = (((int64_t)page * Hkv + g) * page_size + row) * D;
-          for (int d = 0; d < D; ++d)
-            orow[d] += p * kv_elem(v_pages, kv_dtype, dkv_scale, base + d);
+        st = oracle_row(q, k_pages, v_pages, page_table, kv_lens, q_len, Hq, Hkv, D,
+                        page_size, max_pages, num_pages, scale, causal_offset, window,
+                        kv_dtype, kv_scale, tok_lo, tok_hi, b, i, h, s, out, lse);
+        if (st != ORACLE_OK) {
+          free(s);
+          return st;
         }
       }
-    }
-  }
   free(s);
   return ORACLE_OK;
+}
+
+/*
+ * The same rows computed by `threads` OpenMP threads (one row per task; a
+ * row's arithmetic is exactly that of the single-threaded entry point, so
+ * the results are bit-identical). Used to time the oracle on all host cores.
+ * Without OpenMP support at build time it runs single-threaded.
+ */
+int oracle_paged_decode_attn_mt(const uint16_t* q, const void* k_pages,
+                                const void* v_pages, const int32_t* page_table,
+                                const int32_t* kv_lens, int B, int q_len, int Hq,
+                                int Hkv, int D, int page_size, int max_pages,
+                                int num_pages, float scale, int causal_offset,
+                                int window, int kv_dtype, float kv_scale,
+                                double* out, double* lse, int threads) {
+  int64_t max_len;
+  int st = check_args(kv_lens, B, q_len, Hq, Hkv, D, page_size, max_pages, num_pages,
+                      causal_offset, kv_dtype, &max_len);
+  if (st != ORACLE_OK) return st;
+  const int64_t rows = (int64_t)B * q_len * Hq;
+  int status = ORACLE_OK;
+  if (threads < 1) threads = 1;
+#pragma omp parallel num_threads(threads)
+  {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+    int local = s ? ORACLE_OK : ORACLE_NO_MEMORY;
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+      if (local != ORACLE_OK) continue;
+      const int h = (int)(r % Hq);
+      const int i = (int)((r / Hq) % q_len);
+      const int b = (int)(r / ((int64_t)Hq * q_len));
+      local = oracle_row(q, k_pages, v_pages, page_table, kv_lens, q_len, Hq, Hkv, D,
+                         page_size, max_pages, num_pages, scale, causal_offset, window,
+                         kv_dtype, kv_scale, 0, -1, b, i, h, s, out, lse);
+    }
+#pragma omp critical
+    if (local != ORACLE_OK) status = local;
+    free(s);
+  }
+  return status;
+}
+
+/* Number of threads an OpenMP parallel region would use (1 without OpenMP). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
 }
 
 /*

@@ -34,7 +34,7 @@ def build(out_path: str = _LIB_PATH, extra_flags=()) -> str:
     IEEE double operation.
     """
     cmd = [
-        "gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-Wall",
+        "gcc", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared", "-Wall",
         *extra_flags, _SRC, "-o", out_path, "-lm",
     ]
     subprocess.run(cmd, check=True)
@@ -75,6 +75,15 @@ def _declare(lib):
         ctypes.c_int64, ctypes.c_int64,     # tok_lo, tok_hi
         p, p,                               # out, lse
     ]
+    lib.oracle_paged_decode_attn_mt.restype = i32
+    lib.oracle_paged_decode_attn_mt.argtypes = [
+        p, p, p, p, p,
+        i32, i32, i32, i32, i32, i32, i32, i32,
+        ctypes.c_float, i32, i32, i32, ctypes.c_float,
+        p, p, i32,                          # out, lse, threads
+    ]
+    lib.oracle_max_threads.restype = i32
+    lib.oracle_max_threads.argtypes = []
     lib.oracle_merge_states.restype = i32
     lib.oracle_merge_states.argtypes = [p, p, i32, ctypes.c_int64, i32, p, p]
     return lib
@@ -95,13 +104,15 @@ def e4m3_to_double(code: int, lib=None) -> float:
 def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
                       num_kv_heads, page_size, scale, causal_offset=CAUSAL_OFF,
                       window=0, kv_dtype=ORACLE_KV_BF16, kv_scale=1.0,
-                      tok_range=None, lib=None):
+                      tok_range=None, threads=1, lib=None):
     """Run the oracle on host arrays.
 
     q_bits      uint16 [B, q_len, Hq, D]   (bf16 bit patterns)
     k/v_pages   uint16 or uint8 [num_pages, Hkv, page_size, D]
     page_table  int32 [B, max_pages];  kv_lens int32 [B]
     tok_range   optional (lo, hi): keep only keys with lo <= j < hi
+    threads     > 1: the same rows on that many OpenMP threads (bit-identical
+                results; no tok_range)
     Returns (out float64 [B, q_len, Hq, D], lse float64 [B, q_len, Hq]).
     """
     lib = lib or load()
@@ -119,6 +130,17 @@ def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
     out = np.zeros((B, q_len, Hq, D), dtype=np.float64)
     lse = np.zeros((B, q_len, Hq), dtype=np.float64)
     lo, hi = (0, -1) if tok_range is None else tok_range
+    if threads > 1:
+        if tok_range is not None:
+            raise ValueError("tok_range is only supported single-threaded")
+        rc = lib.oracle_paged_decode_attn_mt(
+            _ptr(q_bits), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+            _ptr(kv_lens), B, q_len, Hq, num_kv_heads, D, page_size, max_pages,
+            num_pages, float(scale), int(causal_offset), int(window),
+            int(kv_dtype), float(kv_scale), _ptr(out), _ptr(lse), int(threads))
+        if rc != 0:
+            raise ValueError(f"oracle_paged_decode_attn_mt failed with status {rc}")
+        return out, lse
     rc = lib.oracle_paged_decode_attn(
         _ptr(q_bits), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
         _ptr(kv_lens), B, q_len, Hq, num_kv_heads, D, page_size, max_pages,
@@ -127,6 +149,11 @@ def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
     if rc != 0:
         raise ValueError(f"oracle_paged_decode_attn failed with status {rc}")
     return out, lse
+
+
+def max_threads(lib=None) -> int:
+    """OpenMP threads the multi-threaded entry point uses by default."""
+    return int((lib or load()).oracle_max_threads())
 
 
 def merge_states(o_parts, lse_parts, lib=None):

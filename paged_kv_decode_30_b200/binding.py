@@ -21,6 +21,7 @@ PDA_CAUSAL_OFF = -1
 PDA_CAUSAL_BOTTOM_RIGHT = -2
 PDA_FLAG_NO_PDL = 1
 PDA_FLAG_TENSOR_CORES = 2
+PDA_FLAG_CUDA_CORES = 4
 # Size of the library's fixed partials array used by paged_decode_attn_no_alloc.
 PDA_NO_ALLOC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
@@ -34,8 +35,11 @@ STATUS = {
 EXPORTED = (
     "paged_decode_attn", "paged_decode_attn_no_alloc", "paged_decode_attn_workspace_bytes",
     "pda_choose_num_splits", "pda_merge_states", "pda_status_string",
-    "pda_last_device_error", "pda_abi_version",
+    "pda_last_device_error", "pda_abi_version", "pda_plan_kernel", "pda_hbm_read_probe",
 )
+PDA_KERNEL_SPLIT_FMA = 0
+PDA_KERNEL_SPLIT_TMA = 1
+KERNEL_NAMES = {PDA_KERNEL_SPLIT_FMA: "split_fma_kernel", PDA_KERNEL_SPLIT_TMA: "split_tma_kernel"}
 
 
 class PdaError(RuntimeError):
@@ -102,6 +106,10 @@ def load(path: Optional[str] = None):
     lib.pda_last_device_error.argtypes = [vp]
     lib.pda_abi_version.restype = i32
     lib.pda_abi_version.argtypes = []
+    lib.pda_plan_kernel.restype = i32
+    lib.pda_plan_kernel.argtypes = [pp]
+    lib.pda_hbm_read_probe.restype = i32
+    lib.pda_hbm_read_probe.argtypes = [vp, ctypes.c_size_t, vp, vp]
     if path is None:
         _lib = lib
     return lib
@@ -131,6 +139,20 @@ def status_string(status: int) -> str:
 
 def choose_num_splits(params: PdaParams, num_sms: int) -> int:
     return load().pda_choose_num_splits(ctypes.byref(params), num_sms)
+
+
+def plan_kernel(params: PdaParams) -> int:
+    """PDA_KERNEL_SPLIT_FMA or PDA_KERNEL_SPLIT_TMA (-1: invalid params)."""
+    return load().pda_plan_kernel(ctypes.byref(params))
+
+
+def hbm_read_probe(buf, sink, stream=None):
+    """Read every byte of the CUDA tensor ``buf`` once (bandwidth probe);
+    ``sink`` is an 8-byte CUDA tensor the kernel XORs into."""
+    st = load().pda_hbm_read_probe(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink),
+                                   _stream_handle(stream))
+    if st != 0:
+        raise PdaError(st, "pda_hbm_read_probe")
 
 
 def workspace_bytes(params: PdaParams) -> int:

@@ -16,7 +16,6 @@
 
 #include "merge.cuh"
 #include "paged_decode_attn.h"
-#include "split_tc.cuh"
 #include "split_tma.cuh"
 #include "split_variants.cuh"
 
@@ -85,13 +84,20 @@ bool pool_rows_fit(const pda_params* p) {
   return (long long)p->num_pages * p->num_kv_heads * p->page_size < (1ll << 31);
 }
 
-// The tensor-core kernel takes FP8 K/V with head_dim 128 when the packed
-// rows of a kv head (G * q_len) exceed what the FMA kernel holds in one CTA
-// (8): then QK^T and PV are real dense contractions (N = 16 or 32 rows).
+// Kernel choice for head_dim 128 (the tensor-core kernel's only width):
+//  - FP8 K/V with more than 8 packed rows per kv head (G * q_len): QK^T and
+//    PV are dense contractions with N = 16 or 32 rows;
+//  - bf16 K/V with at most 8 packed rows: one CTA per (b, kv head) streams
+//    the K/V tiles by TMA and hands the contractions to tcgen05, which keeps
+//    the SMs' issue slots (and power) free; measured faster than the FMA
+//    kernel at both full and power-capped clocks on the long-context bf16
+//    workloads.
+// The flags force either kernel.
 bool use_tensor_cores(const pda_params* p, int M) {
   if (p->head_dim != 128 || p->page_size < 8 || !pool_rows_fit(p)) return false;
-  if (p->kv_dtype == PDA_KV_FP8_E4M3) return M > 8;
-  return (p->flags & PDA_FLAG_TENSOR_CORES) != 0;  // bf16: opt-in
+  if (p->flags & PDA_FLAG_CUDA_CORES) return false;
+  if (p->flags & PDA_FLAG_TENSOR_CORES) return true;
+  return p->kv_dtype == PDA_KV_FP8_E4M3 ? M > 8 : M <= 8;
 }
 
 pda_status validate(const pda_params* p) {
@@ -220,6 +226,11 @@ const char* pda_status_string(pda_status s) {
     case PDA_ERR_TIMEOUT: return "device wait timed out";
     default: return "unknown status";
   }
+}
+
+int32_t pda_plan_kernel(const pda_params* params) {
+  if (validate(params) != PDA_OK) return -1;
+  return make_plan(params).tc ? PDA_KERNEL_SPLIT_TMA : PDA_KERNEL_SPLIT_FMA;
 }
 
 int32_t pda_choose_num_splits(const pda_params* params, int32_t num_sms) {

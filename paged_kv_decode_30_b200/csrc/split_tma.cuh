@@ -41,7 +41,7 @@
 
 #include "pda_device.cuh"
 #include "split_fma.cuh"  // SplitArgs, row_range
-#include "split_tc.cuh"   // umma helpers
+#include "tcgen05.cuh"    // descriptors, MMA issue, TMEM loads, barriers
 
 namespace pda {
 
@@ -86,7 +86,11 @@ struct TmaCfg {
   static constexpr int OFF_INV = OFF_LRED + 4 * 32 * 4;  // v_scale / l per row
   static constexpr int OFF_ROWS = OFF_INV + 32 * 4;      // output row of each packed row
   static constexpr int OFF_RANGE = OFF_ROWS + 32 * 8;
-  static constexpr int OFF_BAR = OFF_RANGE + 32 * 8;
+  // page ids of upcoming tiles: PID_SLOTS tiles x 16 segments, filled by
+  // cp.async PID_AHEAD tiles ahead of the copies that use them
+  static constexpr int PID_SLOTS = 8, PID_AHEAD = 4;
+  static constexpr int OFF_PIDS = OFF_RANGE + 32 * 8;
+  static constexpr int OFF_BAR = OFF_PIDS + PID_SLOTS * 16 * 4;
   // full[S], empty[S], s_full[2], p_ready[2], o_full[2], o_free[2], v_ready[2]
   static constexpr int NUM_BARS = 2 * STAGES + 10;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
@@ -230,23 +234,41 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
     const int first = ((kfirst + n) * C::TILE) >> a.log2_page;
     return a.page_size >= C::TILE ? 1 : min(C::TILE >> a.log2_page, seq_pages - first);
   };
-  auto load_pid = [&](int n) -> int {
-    if (n >= ntiles || lane >= nseg_of(n)) return 0;
-    int pid = __ldg(pt_row + (((kfirst + n) * C::TILE) >> a.log2_page) + lane);
+  // Page ids reach shared memory by 4-byte cp.async, one commit group per
+  // tile, PID_AHEAD tiles before they are used: the producer never waits on
+  // a global load of the page table (a register hand-off would stall on the
+  // load's full latency every tile).
+  int32_t* sm_pids = reinterpret_cast<int32_t*>(smem + C::OFF_PIDS);
+  auto prefetch_pids = [&](int n) {
+    if (n < ntiles && lane < nseg_of(n)) {
+      const int32_t* src = pt_row + (((kfirst + n) * C::TILE) >> a.log2_page) + lane;
+      const uint32_t dst = smem_addr(sm_pids + (n % C::PID_SLOTS) * 16 + lane);
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  auto read_pid = [&](int n) -> int {  // after tile n's group completed
+    if (lane >= nseg_of(n)) return 0;
+    int pid = sm_pids[(n % C::PID_SLOTS) * 16 + lane];
     if ((unsigned)pid >= (unsigned)a.num_pages) {
       record_error_at(a.err, kErrBadPage);
       pid = 0;
     }
     return pid;
   };
-  int p_issued = 0, pid_cur = 0;
+  int p_issued = 0;
   // Issue tiles [p_issued, n_end): wait for the stage to be free, set the
   // transaction count, then lane g copies segment g (K and V, both halves
   // of each row for bf16) so the copies of a tile go out together.
   auto produce = [&](int n_end) {
     const uint32_t sbase = smem_addr(smem);
     for (int n = p_issued; n < n_end; ++n) {
-      const int pid_nxt = load_pid(n + 1);  // in flight while we wait
+      // groups complete in order: at most PID_AHEAD - 1 younger than tile n
+      asm volatile("cp.async.wait_group %0;" ::"n"(C::PID_AHEAD - 1) : "memory");
+      __syncwarp();
+      const int pid_cur = read_pid(n);
+      __syncwarp();  // slot n % PID_SLOTS is read before it can be refilled
+      prefetch_pids(n + C::PID_AHEAD);
       const int st = n % C::STAGES;
       bool ok = !*abort_flag;
       if (ok && n >= C::STAGES) ok = mbar_wait(&empty[st], ((n / C::STAGES) - 1) & 1, a.err);
@@ -273,7 +295,6 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
         }
       }
       p_issued = n + 1;
-      pid_cur = pid_nxt;
     }
   };
   if (warp == 0) {
@@ -285,7 +306,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmk) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmv) : "memory");
       }
-      pid_cur = load_pid(0);
+      for (int n = 0; n < C::PID_AHEAD; ++n) prefetch_pids(n);
       produce(min(C::STAGES, ntiles));
     }
   }
@@ -417,6 +438,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
     // ======================= TMA producer (whole warp) ======================
     // Tiles [0, STAGES) went out before the CTA-wide barrier.
     produce(ntiles);
+    asm volatile("cp.async.wait_all;" ::: "memory");  // none left in flight at exit
     if (lane == 0 && *abort_flag) {
       for (int n = max(0, p_issued - C::STAGES); n < p_issued; ++n)
         mbar_wait(&full[n % C::STAGES], (n / C::STAGES) & 1, a.err, kWaitTimeoutCycles / 16);

@@ -159,3 +159,22 @@ def test_workspace_bytes(lib):
     assert got >= expect_o + 4 * rows * 4 and got < expect_o + 4 * rows * 4 + 512
     assert B.workspace_bytes(headline_params(num_splits=1)) == 0
     assert B.workspace_bytes(headline_params(head_dim=96)) == ctypes.c_size_t(-1).value
+
+
+def test_plan_kernel(lib):
+    """Which split kernel the planner picks: tensor cores for FP8 K/V at
+    head_dim 128 with more than 8 packed rows, bf16 only on request."""
+    fp8 = dict(batch=64, q_len=4, num_q_heads=64, num_kv_heads=8, head_dim=128,
+               page_size=128, max_pages_per_seq=256, num_pages=4096, scale=0.088,
+               kv_dtype=B.PDA_KV_FP8_E4M3, kv_scale=0.01)
+    assert B.plan_kernel(B.make_params(**fp8)) == B.PDA_KERNEL_SPLIT_TMA
+    assert B.plan_kernel(B.make_params(**{**fp8, "q_len": 1})) == B.PDA_KERNEL_SPLIT_FMA
+    assert B.plan_kernel(B.make_params(**{**fp8, "head_dim": 64})) == B.PDA_KERNEL_SPLIT_FMA
+    assert B.plan_kernel(B.make_params(**fp8, flags=B.PDA_FLAG_CUDA_CORES)) == B.PDA_KERNEL_SPLIT_FMA
+    assert B.plan_kernel(B.make_params(**{**fp8, "q_len": 1},
+                                       flags=B.PDA_FLAG_TENSOR_CORES)) == B.PDA_KERNEL_SPLIT_TMA
+    assert B.plan_kernel(headline_params()) == B.PDA_KERNEL_SPLIT_TMA
+    assert B.plan_kernel(headline_params(flags=B.PDA_FLAG_CUDA_CORES)) == B.PDA_KERNEL_SPLIT_FMA
+    assert B.plan_kernel(headline_params(num_q_heads=128)) == B.PDA_KERNEL_SPLIT_FMA  # 16 rows
+    assert B.plan_kernel(headline_params(head_dim=64)) == B.PDA_KERNEL_SPLIT_FMA
+    assert B.plan_kernel(headline_params(head_dim=96)) == -1

@@ -150,3 +150,13 @@ def test_planted_mistake_is_caught(tmp_path, name):
     mlib = orc.load(str(so))
     with pytest.raises(AssertionError):
         pins.run_all(mlib)
+
+
+@pytest.mark.parametrize("wl", [pins.SMALL_CASES[3], pins.SMALL_CASES[6]], ids=lambda w: w.name)
+def test_multithreaded_oracle_is_bit_identical(lib, wl):
+    """The OpenMP entry point (used to time the oracle on all host cores)
+    runs the single-threaded row routine per row: identical bits."""
+    inp = W.generate(wl, device="cpu")
+    ref = pins.run_oracle(inp, lib)
+    got = pins.run_oracle(inp, lib, threads=4)
+    assert np.array_equal(ref[0], got[0]) and np.array_equal(ref[1], got[1])

@@ -89,17 +89,21 @@ def test_parity_vs_oracle(lib, case, splits):
     U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, f"{case.name}/s={splits}")
 
 
-TC_BF16_CASES = [c for c in CASES if c.kv_dtype == BF16 and c.head_dim == 128]
+# head_dim-128 cases: the planner picks the tensor-core kernel for some, the
+# CUDA-core kernel for others; each is also run through the other kernel.
+D128_CASES = [c for c in CASES if c.head_dim == 128]
 
 
-@pytest.mark.parametrize("case", TC_BF16_CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("case", D128_CASES, ids=lambda w: w.name)
 @pytest.mark.parametrize("splits", [0, 1, 3, 64])
-def test_parity_tensor_core_bf16(lib, case, splits):
-    """bf16 K/V through the tensor-core kernel (opt-in flag)."""
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+def test_parity_forced_kernel(lib, case, splits, kernel):
+    """Both split kernels on every head_dim-128 case (flags force the choice)."""
+    flags = B.PDA_FLAG_CUDA_CORES if kernel == "cuda_cores" else B.PDA_FLAG_TENSOR_CORES
     inp = W.generate(case)
     ref_out, ref_lse = U.run_oracle(inp)
-    out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=B.PDA_FLAG_TENSOR_CORES)
-    U.assert_parity(out, lse, ref_out, ref_lse, BF16, f"{case.name}/tc/s={splits}")
+    out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=flags)
+    U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, f"{case.name}/{kernel}/s={splits}")
 
 
 @pytest.mark.parametrize("case", [CASES[2], CASES[5], CASES[7]], ids=lambda w: w.name)
@@ -208,13 +212,15 @@ def test_full_size_sampled(lib, name, seqs):
     assert np.isfinite(out).all()
 
 
-def test_full_size_headline_tensor_core_bf16(lib):
+def test_full_size_headline_cuda_core_kernel(lib):
+    """The headline shape through the CUDA-core kernel (the planner picks the
+    tensor-core kernel there)."""
     case = W.HEADLINE
     inp = W.generate(case, device="cuda")
-    out, lse, _ = U.run_cuda(inp, flags=B.PDA_FLAG_TENSOR_CORES)
+    out, lse, _ = U.run_cuda(inp, flags=B.PDA_FLAG_CUDA_CORES)
     seqs = [3, 64, 126]
     ref_out, ref_lse = U.run_oracle(inp, seqs=seqs)
-    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, BF16, "headline/tc")
+    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, BF16, "headline/cuda_cores")
 
 
 @pytest.mark.parametrize("name", [W.VARLEN.name, W.LONGCTX.name])

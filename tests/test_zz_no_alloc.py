@@ -53,7 +53,8 @@ def test_no_alloc_matches_regular_entry_point_two_calls_in_a_row():
 def test_no_alloc_rejects_partials_beyond_its_limit():
     inp = W.generate(CASE_A)
     t = U.to_device(inp)
-    # 16 splits of 128 * 32 rows of 129 floats (about 34 MB) do not fit
+    # 16 splits of 128 * 32 rows of 129 floats (about 34 MB) do not fit (the
+    # CUDA-core kernel splits 256 keys 16 ways; 128-key tiles would not)
     big = W.Workload(name="no_alloc_big", batch=128, num_q_heads=32, num_kv_heads=8,
                      head_dim=128, page_size=16, kv_lens=("const", 256), seed=43)
     binp = W.generate(big)
@@ -61,12 +62,12 @@ def test_no_alloc_rejects_partials_beyond_its_limit():
     need = B.workspace_bytes(B.make_params(
         batch=128, q_len=1, num_q_heads=32, num_kv_heads=8, head_dim=128, page_size=16,
         max_pages_per_seq=bt["page_table"].shape[1], num_pages=bt["k_pages"].shape[0],
-        scale=W.scale_of(big), num_splits=16))
+        scale=W.scale_of(big), num_splits=16, flags=B.PDA_FLAG_CUDA_CORES))
     assert need > B.PDA_NO_ALLOC_WORKSPACE_BYTES
     with pytest.raises(B.PdaError) as e:
         B.paged_decode_attn_no_alloc(bt["q"], bt["k_pages"], bt["v_pages"], bt["page_table"],
                                      bt["kv_lens"], num_kv_heads=8, scale=W.scale_of(big),
-                                     num_splits=16)
+                                     num_splits=16, flags=B.PDA_FLAG_CUDA_CORES)
     assert e.value.status == 4  # PDA_ERR_WORKSPACE
     # the small case still works afterwards
     out, lse, _ = B.paged_decode_attn_no_alloc(
