@@ -54,6 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fused-merge", action="store_true",
+                    help="tensor-core kernel: merge splits in the kernel (no merge launch)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the read-only HBM probe and the CUDA-graph replay (profiling runs)")
     return ap.parse_args(argv)
@@ -339,6 +341,8 @@ def run_ours(args, rank, world, local):
     lse = torch.empty((wl.batch, wl.q_len, wl.num_q_heads), dtype=torch.float32, device=dev)
     flags = {"auto": 0, "tensor_cores": B.PDA_FLAG_TENSOR_CORES,
              "cuda_cores": B.PDA_FLAG_CUDA_CORES}[args.kernel]
+    if args.fused_merge:
+        flags |= B.PDA_FLAG_FUSED_MERGE
     kw = dict(num_kv_heads=wl.num_kv_heads, scale=scale, causal_offset=wl.causal_offset,
               window=wl.window, kv_scale=inp["kv_scale"], max_kv_len=max_len,
               num_splits=args.splits, flags=flags)

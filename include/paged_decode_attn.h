@@ -81,6 +81,9 @@ typedef enum {
 #define PDA_FLAG_TENSOR_CORES 2u /* use the tensor-core kernel wherever it applies
                                     (head_dim 128), not only where the planner picks it */
 #define PDA_FLAG_CUDA_CORES 4u   /* always use the CUDA-core (FMA) kernel */
+#define PDA_FLAG_FUSED_MERGE 8u  /* tensor-core kernel with splits: the split that
+                                    finishes last for a group of rows merges them
+                                    in the kernel (no merge launch) */
 
 typedef struct {
   int32_t batch;            /* B >= 0 */
@@ -100,7 +103,7 @@ typedef struct {
                                Used only to choose the split count. */
   int32_t num_splits;       /* 0 -> heuristic; > 0 forces this many KV splits */
   uint32_t flags;           /* PDA_FLAG_* */
-  void* workspace;          /* device scratch for split partials, or NULL */
+  void* workspace;          /* device scratch (any contents), or NULL */
   size_t workspace_bytes;   /* size of workspace */
   int32_t* num_splits_out;  /* optional host out: split count used */
 } pda_params;
@@ -125,13 +128,18 @@ typedef struct {
  * and out must be 16-byte aligned; page_table, kv_lens and lse 4-byte
  * aligned; a caller workspace 256-byte aligned (else PDA_ERR_MISALIGNED).
  *
- * Workspace: when the call splits the KV range (num_splits > 1) it needs
- * paged_decode_attn_workspace_bytes(params) bytes of device scratch. If
- * params->workspace is NULL the library uses a grow-only buffer it owns, one
- * per device, shared by every call on that device: calls that may overlap on
- * different streams must pass their own workspace. The library never
- * clears the workspace; every slot the kernels read was written earlier in
- * the same call.
+ * Workspace: paged_decode_attn_workspace_bytes(params) bytes of device
+ * scratch. It holds the split partials when the call splits the KV range,
+ * and, for the tensor-core kernel (see pda_plan_kernel), a header of
+ * counters: the work queue of its persistent CTAs and, per (sequence, kv
+ * head, row tile), how many splits have finished (the last one merges).
+ * The call zeroes that header itself (one small memset on `stream` before
+ * the launch), so the workspace's contents before the call do not matter
+ * and a call captured in a CUDA graph replays correctly. Every partial slot
+ * a kernel reads was written earlier in the same call. If params->workspace is NULL the library
+ * uses a grow-only buffer it owns, one per device, shared by every call on
+ * that device: calls that may overlap on different streams must pass their
+ * own workspace (the same holds for a caller workspace).
  *
  * Errors: invalid sizes or pointers return before any device work. A page
  * id >= num_pages or < 0 met on the device is never dereferenced; the kernel
@@ -181,8 +189,8 @@ PDA_API pda_status paged_decode_attn_no_alloc(const void* q, const void* k_pages
                                               float* lse, pda_stream_t stream);
 
 /* Bytes of workspace paged_decode_attn needs for these params with the
- * split count it would choose (0 when it would not split). SIZE_MAX if the
- * params are invalid. */
+ * split count it would choose (0 for the CUDA-core kernel when it would not
+ * split). SIZE_MAX if the params are invalid. */
 PDA_API size_t paged_decode_attn_workspace_bytes(const pda_params* params);
 
 /* The split count paged_decode_attn would use for these params on a device

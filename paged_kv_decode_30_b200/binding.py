@@ -22,6 +22,7 @@ PDA_CAUSAL_BOTTOM_RIGHT = -2
 PDA_FLAG_NO_PDL = 1
 PDA_FLAG_TENSOR_CORES = 2
 PDA_FLAG_CUDA_CORES = 4
+PDA_FLAG_FUSED_MERGE = 8
 # Size of the library's fixed partials array used by paged_decode_attn_no_alloc.
 PDA_NO_ALLOC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
@@ -177,8 +178,8 @@ def paged_decode_attn(q, k_pages, v_pages, page_table, kv_lens, *, num_kv_heads,
 
     q [B, q_len, Hq, D] bf16; k/v_pages [num_pages, Hkv, P, D] bf16 or uint8
     (e4m3 codes); page_table int32 [B, max_pages]; kv_lens int32 [B].
-    ``workspace``: a CUDA uint8 tensor, or None to let the binding allocate
-    exactly what the call needs.
+    ``workspace``: a CUDA uint8 tensor (any contents; reusable across calls),
+    or None to let the binding allocate exactly what the call needs.
     """
     import torch
     lib = load()

@@ -174,11 +174,32 @@ int choose_splits(const pda_params* p, const Plan& pl, int num_sms) {
   return best;
 }
 
-size_t partial_bytes(const Plan& pl, int splits, int D, size_t* lse_offset) {
-  const size_t o_bytes = (size_t)splits * (size_t)pl.rows * (size_t)D * sizeof(float);
-  const size_t off = (o_bytes + 255) / 256 * 256;
-  if (lse_offset) *lse_offset = off;
-  return off + (size_t)splits * (size_t)pl.rows * sizeof(float);
+// Workspace layout. The tensor-core kernel keeps its work-queue counter and
+// one split-arrival counter per (sequence, kv head, row tile) at the front
+// (zeroed by a memset on the call's stream before the launch); the split
+// partials follow (o_part then lse_part).
+struct WsLayout {
+  size_t counters;  // bytes of the counter header (0 for the FMA kernel)
+  size_t o_off, lse_off, total;
+};
+constexpr size_t kMergeCtrOffset = 64;  // bytes: after the work-queue counters
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+
+WsLayout ws_layout(const pda_params* p, const Plan& pl, int splits) {
+  WsLayout w{};
+  if (pl.tc) {
+    const size_t groups = (size_t)p->batch * (size_t)p->num_kv_heads * (size_t)pl.row_tiles;
+    w.counters = round256(kMergeCtrOffset + groups * sizeof(int));
+  }
+  w.o_off = w.lse_off = w.total = w.counters;
+  if (splits > 1) {
+    const size_t o_bytes = (size_t)splits * (size_t)pl.rows * (size_t)p->head_dim * sizeof(float);
+    w.lse_off = w.o_off + round256(o_bytes);
+    w.total = w.lse_off + (size_t)splits * (size_t)pl.rows * sizeof(float);
+  }
+  return w;
 }
 
 }  // namespace
@@ -245,7 +266,7 @@ size_t paged_decode_attn_workspace_bytes(const pda_params* params) {
   DeviceState* st = nullptr;
   if (params->num_splits == 0 && device_state(&st) == PDA_OK) sms = st->num_sms;
   const int s = choose_splits(params, pl, sms);
-  return s > 1 ? partial_bytes(pl, s, params->head_dim, nullptr) : 0;
+  return ws_layout(params, pl, s).total;
 }
 
 pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_pages,
@@ -304,44 +325,63 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   a.head_stride = (long long)p.page_size * p.head_dim * pl.elt;
   a.page_stride = a.head_stride * p.num_kv_heads;
 
-  if (splits > 1) {
-    size_t lse_off = 0;
-    const size_t need = partial_bytes(pl, splits, p.head_dim, &lse_off);
+  const WsLayout wl = ws_layout(&p, pl, splits);
+  if (wl.total > 0) {
     void* ws = p.workspace;
     if (ws == nullptr) {
       std::lock_guard<std::mutex> lock(g_mu);
-      if (dev->ws_bytes < need) {
+      if (dev->ws_bytes < wl.total) {
         if (dev->ws) cudaFree(dev->ws);  // synchronises the device
         dev->ws = nullptr;
         dev->ws_bytes = 0;
-        if (cudaMalloc(&dev->ws, need) != cudaSuccess) {
+        if (cudaMalloc(&dev->ws, wl.total) != cudaSuccess) {
           dev->ws = nullptr;
           return PDA_ERR_WORKSPACE;
         }
-        dev->ws_bytes = need;
+        dev->ws_bytes = wl.total;
       }
       ws = dev->ws;
-    } else if (p.workspace_bytes < need) {
+    } else if (p.workspace_bytes < wl.total) {
       return PDA_ERR_WORKSPACE;
     }
-    a.o_part = static_cast<float*>(ws);
-    a.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + lse_off);
+    char* base = static_cast<char*>(ws);
+    if (pl.tc) {
+      a.sched = reinterpret_cast<int*>(base);
+      a.merge_ctr = reinterpret_cast<int*>(base + kMergeCtrOffset);
+      // the counters start at zero for this call
+      const size_t used = kMergeCtrOffset +
+          (size_t)p.batch * p.num_kv_heads * pl.row_tiles * sizeof(int);
+      if (cudaMemsetAsync(base, 0, used, stream) != cudaSuccess) return PDA_ERR_CUDA;
+    }
+    if (splits > 1) {
+      a.o_part = reinterpret_cast<float*>(base + wl.o_off);
+      a.lse_part = reinterpret_cast<float*>(base + wl.lse_off);
+    }
   }
 
-  const dim3 grid((unsigned)pl.row_tiles, (unsigned)(splits * p.num_kv_heads), (unsigned)p.batch);
   cudaError_t e;
   const int kv = fp8 ? 1 : 0;
   if (pl.tc) {
+    // persistent: at most one CTA per SM, items from the work queue; the
+    // split that finishes last for a group of rows merges it (no merge launch)
+    const long long items = (long long)p.batch * p.num_kv_heads * splits * pl.row_tiles;
+    if (items > INT_MAX) return PDA_ERR_UNSUPPORTED;
+    a.num_items = (int)items;
+    a.fused_merge = (p.flags & PDA_FLAG_FUSED_MERGE) != 0;
+    const int grid = (int)std::min<long long>(items, dev->num_sms);
     e = launch_split_tma(kv, pl.mt, k_pages, v_pages, a, grid, stream);
-  } else switch (p.head_dim) {
-    case 64: e = launch_split_d64(kv, pl.mt, pl.tw, a, grid, stream); break;
-    case 128: e = launch_split_d128(kv, pl.mt, pl.tw, a, grid, stream); break;
-    case 256: e = launch_split_d256(kv, pl.mt, pl.tw, a, grid, stream); break;
-    default: e = cudaErrorNotSupported;
+  } else {
+    const dim3 grid((unsigned)pl.row_tiles, (unsigned)(splits * p.num_kv_heads), (unsigned)p.batch);
+    switch (p.head_dim) {
+      case 64: e = launch_split_d64(kv, pl.mt, pl.tw, a, grid, stream); break;
+      case 128: e = launch_split_d128(kv, pl.mt, pl.tw, a, grid, stream); break;
+      case 256: e = launch_split_d256(kv, pl.mt, pl.tw, a, grid, stream); break;
+      default: e = cudaErrorNotSupported;
+    }
   }
   if (e == cudaErrorNotSupported) return PDA_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return PDA_ERR_CUDA;
-  if (splits > 1) {
+  if (splits > 1 && !(pl.tc && a.fused_merge)) {
     e = launch_merge(p.head_dim, a.o_part, a.lse_part, splits, pl.rows, out, lse, stream,
                      (p.flags & PDA_FLAG_NO_PDL) == 0);
     if (e != cudaSuccess) return PDA_ERR_CUDA;

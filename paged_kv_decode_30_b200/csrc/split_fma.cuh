@@ -70,6 +70,12 @@ struct SplitArgs {
   float v_scale;             // 1, or kv_scale for FP8
   long long page_stride;     // bytes per page: Hkv * P * D * elt
   long long head_stride;     // bytes per (page, head) block: P * D * elt
+  // persistent tensor-core kernel only (counters zeroed by the host just
+  // before the launch, in stream order):
+  int* sched;                // [0] next work item
+  int* merge_ctr;            // [B * Hkv * row_tiles] splits finished per group
+  int num_items;             // B * Hkv * num_splits * row_tiles
+  int fused_merge;           // 1: the last split of a group merges it in-kernel
 };
 
 template <int D, int KV, int MT, int TW, int NW, int STAGES>

@@ -47,7 +47,7 @@ bool make_pool_map(CUtensorMap* map, const void* base, long long rows, int elt, 
 
 template <int KV, int NT>
 cudaError_t launch_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const SplitArgs& a,
-                       dim3 grid, cudaStream_t stream) {
+                       int grid, cudaStream_t stream) {
   using C = TmaCfg<KV, NT>;
   auto kern = split_tma_kernel<KV, NT>;
   static unsigned long long attr_set = 0;  // bit d: opt-in set on device d (< 64)
@@ -60,14 +60,14 @@ cudaError_t launch_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const Split
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
   }
-  kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mk, mv, a);
+  kern<<<dim3((unsigned)grid), C::THREADS, C::SMEM_ALLOC, stream>>>(mk, mv, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_split_tma(int kv, int nt, const void* k_pages, const void* v_pages,
-                             const SplitArgs& a, dim3 grid, cudaStream_t stream) {
+                             const SplitArgs& a, int grid, cudaStream_t stream) {
   const long long rows = (long long)a.num_pages * a.Hkv * a.page_size;
   const int elt = kv == 0 ? 2 : 1;
   const int box_rows = a.page_size < 128 ? a.page_size : 128;

@@ -152,12 +152,18 @@ def test_split_planner(lib):
 
 
 def test_workspace_bytes(lib):
-    p = headline_params(num_splits=4)
     rows = 128 * 32
     expect_o = 4 * rows * 128 * 4
-    got = B.workspace_bytes(p)
+    # CUDA-core kernel: the split partials only
+    got = B.workspace_bytes(headline_params(num_splits=4, flags=B.PDA_FLAG_CUDA_CORES))
     assert got >= expect_o + 4 * rows * 4 and got < expect_o + 4 * rows * 4 + 512
-    assert B.workspace_bytes(headline_params(num_splits=1)) == 0
+    assert B.workspace_bytes(headline_params(num_splits=1, flags=B.PDA_FLAG_CUDA_CORES)) == 0
+    # tensor-core kernel: a counter header (the work-queue counter, then one
+    # split-arrival counter per (sequence, kv head, row tile)) before the partials
+    header = (64 + 128 * 8 * 4 + 255) // 256 * 256
+    assert B.workspace_bytes(headline_params(num_splits=1)) == header
+    got = B.workspace_bytes(headline_params(num_splits=4))
+    assert got >= header + expect_o + 4 * rows * 4 and got < header + expect_o + 4 * rows * 4 + 512
     assert B.workspace_bytes(headline_params(head_dim=96)) == ctypes.c_size_t(-1).value
 
 

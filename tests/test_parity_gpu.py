@@ -96,10 +96,12 @@ D128_CASES = [c for c in CASES if c.head_dim == 128]
 
 @pytest.mark.parametrize("case", D128_CASES, ids=lambda w: w.name)
 @pytest.mark.parametrize("splits", [0, 1, 3, 64])
-@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores", "tensor_cores_fused_merge"])
 def test_parity_forced_kernel(lib, case, splits, kernel):
-    """Both split kernels on every head_dim-128 case (flags force the choice)."""
-    flags = B.PDA_FLAG_CUDA_CORES if kernel == "cuda_cores" else B.PDA_FLAG_TENSOR_CORES
+    """Both split kernels on every head_dim-128 case (flags force the choice),
+    the tensor-core one also with the in-kernel merge of its splits."""
+    flags = {"cuda_cores": B.PDA_FLAG_CUDA_CORES, "tensor_cores": B.PDA_FLAG_TENSOR_CORES,
+             "tensor_cores_fused_merge": B.PDA_FLAG_TENSOR_CORES | B.PDA_FLAG_FUSED_MERGE}[kernel]
     inp = W.generate(case)
     ref_out, ref_lse = U.run_oracle(inp)
     out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=flags)
@@ -230,3 +232,63 @@ def test_full_size_all_rows(lib, name):
     out, lse, used = U.run_cuda(inp)
     ref_out, ref_lse = U.run_oracle(inp)
     U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, name)
+
+
+@pytest.mark.parametrize("case", [c for c in CASES if c.name.startswith("tc_fp8")][:2] +
+                         [c for c in CASES if c.kv_dtype == BF16 and c.head_dim == 128][:1],
+                         ids=lambda w: w.name)
+def test_workspace_contents_do_not_matter(lib, case):
+    """The call zeroes the tensor-core kernel's counter header itself: a
+    workspace full of random bytes, reused across calls, gives the same
+    results as a fresh one."""
+    inp = W.generate(case)
+    ref_out, ref_lse = U.run_oracle(inp)
+    params_kw = dict(num_splits=3, flags=B.PDA_FLAG_TENSOR_CORES | B.PDA_FLAG_FUSED_MERGE)
+    t = U.to_device(inp)
+    wl = inp["workload"]
+    need = B.workspace_bytes(B.make_params(
+        batch=wl.batch, q_len=wl.q_len, num_q_heads=wl.num_q_heads,
+        num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, page_size=wl.page_size,
+        max_pages_per_seq=t["page_table"].shape[1], num_pages=t["k_pages"].shape[0],
+        scale=W.scale_of(wl), kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"], **params_kw))
+    ws = torch.randint(0, 256, (need,), dtype=torch.uint8, device="cuda",
+                       generator=torch.Generator(device="cuda").manual_seed(11))
+    for rep in range(3):
+        out, lse, used = B.paged_decode_attn(
+            t["q"], t["k_pages"], t["v_pages"], t["page_table"], t["kv_lens"],
+            num_kv_heads=wl.num_kv_heads, scale=W.scale_of(wl), causal_offset=wl.causal_offset,
+            window=wl.window, kv_scale=inp["kv_scale"], workspace=ws, **params_kw)
+        torch.cuda.synchronize()
+        assert B.last_device_error() == 0
+        U.assert_parity(out.double().cpu().numpy(), lse.double().cpu().numpy(), ref_out, ref_lse,
+                        case.kv_dtype, f"{case.name}/garbage-ws/rep{rep}")
+
+
+def test_cuda_graph_replays(lib):
+    """A call captured in a CUDA graph replays correctly many times (the
+    counter memset is part of the captured work)."""
+    case = [c for c in CASES if c.name.startswith("tc_fp8")][0]
+    inp = W.generate(case)
+    ref_out, ref_lse = U.run_oracle(inp)
+    t = U.to_device(inp)
+    wl = inp["workload"]
+    out = torch.empty((wl.batch, wl.q_len, wl.num_q_heads, wl.head_dim), dtype=torch.float32,
+                      device="cuda")
+    lse = torch.empty((wl.batch, wl.q_len, wl.num_q_heads), dtype=torch.float32, device="cuda")
+    ws = torch.empty(1 << 22, dtype=torch.uint8, device="cuda")
+    kw = dict(num_kv_heads=wl.num_kv_heads, scale=W.scale_of(wl), causal_offset=wl.causal_offset,
+              window=wl.window, kv_scale=inp["kv_scale"], num_splits=2, out=out, lse=lse,
+              workspace=ws, flags=B.PDA_FLAG_FUSED_MERGE)
+    B.paged_decode_attn(t["q"], t["k_pages"], t["v_pages"], t["page_table"], t["kv_lens"], **kw)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        B.paged_decode_attn(t["q"], t["k_pages"], t["v_pages"], t["page_table"], t["kv_lens"], **kw)
+    for rep in range(4):
+        out.fill_(float("nan"))
+        lse.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert B.last_device_error() == 0
+        U.assert_parity(out.double().cpu().numpy(), lse.double().cpu().numpy(), ref_out, ref_lse,
+                        case.kv_dtype, f"graph replay {rep}")
