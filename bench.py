@@ -409,7 +409,8 @@ def run_ours(args, rank, world, local):
     avg_launch_ms = statistics.mean(step_ms)
     achieved = alg_bytes / (avg_launch_ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
-    launches_per_step = 1 + (1 if splits > 1 else 0)
+    merge_launched = splits > 1 and not (kernel_name == "split_tma_kernel" and args.fused_merge)
+    launches_per_step = 1 + (1 if merge_launched else 0)
 
     # Read-only HBM probe in the same run (our streaming-load kernel over a
     # 4 GiB buffer, larger than L2): the ceiling for a kernel that only reads.
@@ -537,7 +538,7 @@ def run_ours(args, rank, world, local):
             "traffic_unit": "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)",
             "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
             "frac_of_8tbs_spec": achieved / 8000.0,
-            "kernel": kernel_name + (" + merge_states_kernel" if splits > 1 else ""),
+            "kernel": kernel_name + (" + merge_states_kernel" if merge_launched else ""),
             "read_probe_gbs": probe_gbs,
             "frac_of_read_probe": achieved / probe_gbs if probe_gbs else None,
             "avg_launch_ms": avg_launch_ms,
