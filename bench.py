@@ -499,6 +499,41 @@ def run_ours(args, rank, world, local):
                "d2h_bytes_per_step": hout.numel() * 4 + hlse.numel() * 4,
                "steps": n_e2e}
 
+    # The KV-cache producer on the same cache (measured after the decode
+    # timing; it overwrites the last slots of each sequence): one new token
+    # per sequence (a decode step's append) and 64 (a chunk's), K and V.
+    kv_append = None
+    if not args.no_extras:
+        kv_append = {}
+        elt = 2 if wl.kv_dtype == W.KV_BF16 else 1
+        for T in (1, 64):
+            if int(kl.min().item()) < T:
+                continue
+            kn = torch.randn((wl.batch, T, wl.num_kv_heads, wl.head_dim), device=dev).to(torch.bfloat16)
+            vn = torch.randn_like(kn)
+            base = (kl - T).contiguous()
+            for _ in range(3):
+                B.paged_kv_append(kn, vn, pt, base, kp, vp, kv_scale=inp["kv_scale"])
+            # 50 appends in one CUDA graph: device time, not Python call rate
+            n_app = 50
+            ga = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga):
+                for _ in range(n_app):
+                    B.paged_kv_append(kn, vn, pt, base, kp, vp, kv_scale=inp["kv_scale"])
+            ga.replay()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            ga.replay()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            del ga
+            ms = a0.elapsed_time(a1) / n_app
+            nbytes = 2 * wl.batch * T * wl.num_kv_heads * wl.head_dim * (2 + elt)
+            kv_append[f"tokens_{T}"] = {"ms": ms, "bytes": nbytes, "gb_s": nbytes / (ms / 1e3) / 1e9,
+                                        "frac_of_copy": nbytes / (ms / 1e3) / 1e9 / peak}
+        if B.last_device_error() != 0:
+            raise RuntimeError("device error word set by the append measurement")
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, args.cpu_seconds)
@@ -546,6 +581,7 @@ def run_ours(args, rank, world, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "graph": graph,
+        "kv_append": kv_append,
         "e2e": e2e,
         "cpu_baseline": cpu,
     }

@@ -216,6 +216,51 @@ PDA_API pda_status pda_merge_states(const float* o_parts, const float* lse_parts
                             int32_t num_splits, int64_t rows, int32_t head_dim,
                             float* out, float* lse, pda_stream_t stream);
 
+/* Parameters of paged_kv_append. */
+typedef struct {
+  int32_t batch;             /* B >= 0 */
+  int32_t num_new;           /* new tokens per sequence, 1..64 */
+  int32_t num_kv_heads;      /* Hkv >= 1 */
+  int32_t head_dim;          /* D in {64, 128, 256} */
+  int32_t page_size;         /* P, a power of two in [8, 256] */
+  int32_t max_pages_per_seq; /* row stride of page_table */
+  int32_t num_pages;         /* pages in each pool; page ids must be < this */
+  int32_t kv_dtype;          /* pda_kv_dtype of the pools */
+  float kv_scale;            /* FP8 only: code = e4m3(x / kv_scale) (> 0) */
+} pda_append_params;
+
+/*
+ * Paged KV append, the KV-cache producer that runs before the decode call
+ * ("sglang profiler skill, fuse-overlap catalog", "Fused FP8 quantize + paged
+ * KV cache write" row): new row t of sequence b (t < num_new) is written at
+ * logical position kv_lens[b] + t, i.e. page page_table[b][pos / P], slot
+ * pos % P, for every kv head, in K and in V.
+ *
+ * k_new, v_new  device, bf16 [B, num_new, Hkv, D], contiguous, 16-byte aligned.
+ * page_table    device, int32 [B, max_pages_per_seq]; the pages covering
+ *               [kv_lens[b], kv_lens[b] + num_new) must already be assigned.
+ * kv_lens       device, int32 [B]: lengths before the append. Read only: the
+ *               caller advances them by num_new before the next decode call.
+ * params        host, read during the call only.
+ * k_pages, v_pages device pools [num_pages, Hkv, P, D] of bf16 or e4m3 codes
+ *               (kv_dtype), 16-byte aligned. Only the appended slots are written.
+ *
+ * bf16 pools receive the bits unchanged. FP8 pools receive, per element, the
+ * e4m3 code nearest to the fp32 quotient x / kv_scale (IEEE division), ties
+ * to even, saturated to +-448 (NaN stays NaN): the encoding the decode call
+ * inverts with the same kv_scale.
+ *
+ * Errors: invalid params or pointers return before any device work
+ * (PDA_ERR_INVALID_ARG / _UNSUPPORTED / _MISALIGNED). A position past
+ * max_pages_per_seq * P, a negative kv_len or a page id out of range is not
+ * written and records PDA_ERR_BAD_PAGE in the device error word.
+ * Asynchronous on `stream`.
+ */
+PDA_API pda_status paged_kv_append(const void* k_new, const void* v_new,
+                                   const int32_t* page_table, const int32_t* kv_lens,
+                                   const pda_append_params* params, void* k_pages,
+                                   void* v_pages, pda_stream_t stream);
+
 /* Which split kernel paged_decode_attn would launch for these params
  * (host-only; the planner's choice):
  *   PDA_KERNEL_SPLIT_TMA  tensor-core kernel (2D TMA tiles of 128 tokens,

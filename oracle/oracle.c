@@ -292,6 +292,79 @@ int oracle_max_threads(void) {
 }
 
 /*
+ * E4M3 encoding of a float, from the format's definition: the finite code
+ * whose value is nearest to x, ties to the code with an even mantissa (even
+ * code), magnitudes of 448 and above (and infinities) saturating to +-448,
+ * NaN to 0x7F. Walks all 127 non-negative codes; no table, no bit tricks.
+ */
+uint8_t oracle_e4m3_encode(float x) {
+  if (isnan(x)) return 0x7F;
+  const int neg = signbit(x) ? 1 : 0;
+  const double a = fabs((double)x);
+  int best = 0;
+  if (a >= 448.0) {
+    best = 0x7E;
+  } else {
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+      const double err = fabs(a - oracle_e4m3_to_double((uint8_t)c));
+      if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+        best_err = err;
+        best = c;
+      }
+    }
+  }
+  return (uint8_t)(best | (neg << 7));
+}
+
+/*
+ * Paged KV append (the KV-cache producer): new row t of sequence b goes to
+ * logical position pos = kv_lens[b] + t, i.e. page page_table[b][pos / P],
+ * slot pos % P, for every kv head. bf16 pools receive the bits unchanged;
+ * FP8 pools receive oracle_e4m3_encode(x / kv_scale), the quotient taken in
+ * single precision (the precision in which the quantised code is decided).
+ *
+ * k_new, v_new  bf16 bits [B, num_new, Hkv, D]
+ * k/v_pages     bf16 bits or e4m3 bytes [num_pages, Hkv, P, D], updated in place
+ * Returns ORACLE_BAD_PAGE (writing nothing more) at the first position past
+ * the page table or page id out of range.
+ */
+int oracle_paged_kv_append(const uint16_t* k_new, const uint16_t* v_new,
+                           const int32_t* page_table, const int32_t* kv_lens, int B,
+                           int num_new, int Hkv, int D, int page_size, int max_pages,
+                           int num_pages, int kv_dtype, float kv_scale, void* k_pages,
+                           void* v_pages) {
+  if (B < 0 || num_new < 1 || Hkv < 1 || D < 1 || page_size < 1 || max_pages < 1 ||
+      num_pages < 1)
+    return ORACLE_BAD_ARG;
+  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3) return ORACLE_BAD_ARG;
+  for (int b = 0; b < B; ++b) {
+    for (int t = 0; t < num_new; ++t) {
+      const int64_t pos = (int64_t)kv_lens[b] + t;
+      if (kv_lens[b] < 0 || pos >= (int64_t)max_pages * page_size) return ORACLE_BAD_PAGE;
+      const int32_t page = page_table[(int64_t)b * max_pages + pos / page_size];
+      if (page < 0 || page >= num_pages) return ORACLE_BAD_PAGE;
+      for (int h = 0; h < Hkv; ++h) {
+        const int64_t src = (((int64_t)b * num_new + t) * Hkv + h) * D;
+        const int64_t dst = (((int64_t)page * Hkv + h) * page_size + pos % page_size) * D;
+        for (int d = 0; d < D; ++d) {
+          if (kv_dtype == ORACLE_KV_BF16) {
+            ((uint16_t*)k_pages)[dst + d] = k_new[src + d];
+            ((uint16_t*)v_pages)[dst + d] = v_new[src + d];
+          } else {
+            const float kx = (float)oracle_bf16_to_double(k_new[src + d]);
+            const float vx = (float)oracle_bf16_to_double(v_new[src + d]);
+            ((uint8_t*)k_pages)[dst + d] = oracle_e4m3_encode(kx / kv_scale);
+            ((uint8_t*)v_pages)[dst + d] = oracle_e4m3_encode(vx / kv_scale);
+          }
+        }
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+/*
  * Log-sum-exp merge of n attention states over disjoint key sets
  * (merge_attn_states / PagedPersistentMergeKernel):
  *   lse = m* + ln sum_s exp(lse_s - m*),  m* = max_s lse_s

@@ -84,6 +84,15 @@ def _declare(lib):
     ]
     lib.oracle_max_threads.restype = i32
     lib.oracle_max_threads.argtypes = []
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_paged_kv_append.restype = i32
+    lib.oracle_paged_kv_append.argtypes = [
+        p, p, p, p,                          # k_new, v_new, page_table, kv_lens
+        i32, i32, i32, i32, i32, i32, i32,   # B num_new Hkv D P max_pages num_pages
+        i32, ctypes.c_float,                 # kv_dtype, kv_scale
+        p, p,                                # k_pages, v_pages (in place)
+    ]
     lib.oracle_merge_states.restype = i32
     lib.oracle_merge_states.argtypes = [p, p, i32, ctypes.c_int64, i32, p, p]
     return lib
@@ -149,6 +158,35 @@ def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
     if rc != 0:
         raise ValueError(f"oracle_paged_decode_attn failed with status {rc}")
     return out, lse
+
+
+def e4m3_encode(x: float, lib=None) -> int:
+    return int((lib or load()).oracle_e4m3_encode(float(x)))
+
+
+def paged_kv_append(k_new_bits, v_new_bits, page_table, kv_lens, k_pages, v_pages, *,
+                    page_size, kv_dtype=ORACLE_KV_BF16, kv_scale=1.0, lib=None):
+    """Append new rows into copies of the pools; returns (k_pages, v_pages).
+
+    k/v_new_bits  uint16 [B, num_new, Hkv, D] (bf16 bit patterns)
+    k/v_pages     uint16 or uint8 [num_pages, Hkv, page_size, D]
+    """
+    lib = lib or load()
+    k_new_bits = np.ascontiguousarray(k_new_bits, dtype=np.uint16)
+    v_new_bits = np.ascontiguousarray(v_new_bits, dtype=np.uint16)
+    kdt = np.uint16 if kv_dtype == ORACLE_KV_BF16 else np.uint8
+    kp = np.array(k_pages, dtype=kdt, copy=True, order="C")
+    vp = np.array(v_pages, dtype=kdt, copy=True, order="C")
+    page_table = np.ascontiguousarray(page_table, dtype=np.int32)
+    kv_lens = np.ascontiguousarray(kv_lens, dtype=np.int32)
+    B, num_new, Hkv, D = k_new_bits.shape
+    rc = lib.oracle_paged_kv_append(
+        _ptr(k_new_bits), _ptr(v_new_bits), _ptr(page_table), _ptr(kv_lens), B, num_new,
+        Hkv, D, page_size, page_table.shape[1], kp.shape[0], int(kv_dtype), float(kv_scale),
+        _ptr(kp), _ptr(vp))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_kv_append failed with status {rc}")
+    return kp, vp
 
 
 def max_threads(lib=None) -> int:

@@ -37,6 +37,7 @@ EXPORTED = (
     "paged_decode_attn", "paged_decode_attn_no_alloc", "paged_decode_attn_workspace_bytes",
     "pda_choose_num_splits", "pda_merge_states", "pda_status_string",
     "pda_last_device_error", "pda_abi_version", "pda_plan_kernel", "pda_hbm_read_probe",
+    "paged_kv_append",
 )
 PDA_KERNEL_SPLIT_FMA = 0
 PDA_KERNEL_SPLIT_TMA = 1
@@ -47,6 +48,22 @@ class PdaError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
         super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class PdaAppendParams(ctypes.Structure):
+    """Mirror of ``pda_append_params``."""
+
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("num_new", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("kv_dtype", ctypes.c_int32),
+        ("kv_scale", ctypes.c_float),
+    ]
 
 
 class PdaParams(ctypes.Structure):
@@ -109,6 +126,8 @@ def load(path: Optional[str] = None):
     lib.pda_abi_version.argtypes = []
     lib.pda_plan_kernel.restype = i32
     lib.pda_plan_kernel.argtypes = [pp]
+    lib.paged_kv_append.restype = i32
+    lib.paged_kv_append.argtypes = [vp, vp, vp, vp, ctypes.POINTER(PdaAppendParams), vp, vp, vp]
     lib.pda_hbm_read_probe.restype = i32
     lib.pda_hbm_read_probe.argtypes = [vp, ctypes.c_size_t, vp, vp]
     if path is None:
@@ -246,6 +265,26 @@ def paged_decode_attn_no_alloc(q, k_pages, v_pages, page_table, kv_lens, *,
     if st != 0:
         raise PdaError(st, "paged_decode_attn_no_alloc")
     return out, lse, used.value
+
+
+def paged_kv_append(k_new, v_new, page_table, kv_lens, k_pages, v_pages, *, kv_scale=1.0,
+                    stream=None):
+    """Write new K/V rows (bf16 [B, num_new, Hkv, D]) into the pools at
+    positions kv_lens[b] + t (kv_lens is not advanced). Pools of uint8 are
+    e4m3 codes quantised with kv_scale; bf16 pools get the bits."""
+    import torch
+    B, T, Hkv, D = k_new.shape
+    kv_dtype = PDA_KV_FP8_E4M3 if k_pages.dtype == torch.uint8 else PDA_KV_BF16
+    for t_ in (k_new, v_new, page_table, kv_lens, k_pages, v_pages):
+        if not t_.is_cuda or not t_.is_contiguous():
+            raise ValueError("all inputs must be contiguous CUDA tensors")
+    p = PdaAppendParams(B, T, Hkv, D, k_pages.shape[2], page_table.shape[1], k_pages.shape[0],
+                        kv_dtype, kv_scale)
+    st = load().paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(page_table), _ptr(kv_lens),
+                                ctypes.byref(p), _ptr(k_pages), _ptr(v_pages),
+                                _stream_handle(stream))
+    if st != 0:
+        raise PdaError(st, "paged_kv_append")
 
 
 def merge_states(o_parts, lse_parts, *, out=None, lse=None, stream=None):

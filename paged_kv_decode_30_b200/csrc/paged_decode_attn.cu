@@ -204,6 +204,13 @@ WsLayout ws_layout(const pda_params* p, const Plan& pl, int splits) {
 
 }  // namespace
 
+// Device address of the current device's error word (nullptr if the device
+// cannot be initialised); used by the other entry points of the library.
+int* device_error_word() {
+  DeviceState* st = nullptr;
+  return device_state(&st) == PDA_OK ? st->err : nullptr;
+}
+
 cudaError_t launch_merge(int D, const float* o_parts, const float* lse_parts,
                          int num_splits, long long rows, float* out, float* lse,
                          cudaStream_t stream, bool pdl) {

@@ -17,6 +17,12 @@ What pins what:
   * closed forms: equal keys -> mean of visible V and lse = s + ln |V|;
     one-hot V -> softmax probabilities; single key -> v.
   * golden: hand-derived fixtures under tests/golden/.
+  * e4m3 encode: inverts torch's decode on every finite code; equals torch's
+    float8_e4m3fn cast (round to nearest even) on 200k log-uniform values and
+    on every exact midpoint between adjacent codes.
+  * append: new rows land where numpy indexing of the page table says
+    (page_table[b][pos // P], slot pos % P), as torch-cast codes for FP8;
+    every other slot is unchanged.
 """
 
 from __future__ import annotations
@@ -323,3 +329,73 @@ def run_all(lib):
     check_equal_keys(lib)
     check_one_hot_values(lib)
     check_poison_is_never_read(SMALL_CASES[3], lib)
+    check_e4m3_encode_roundtrip(lib)
+    check_e4m3_encode_vs_torch(lib, n=20_000)
+    check_append(lib, W.KV_BF16)
+    check_append(lib, W.KV_FP8_E4M3)
+
+
+# ---------------------------------------------------------------------------
+# KV append: e4m3 encoding and the page placement of new rows
+
+def check_e4m3_encode_roundtrip(lib):
+    """encode(decode(c)) == c for every finite code; values decoded by torch."""
+    codes = torch.tensor([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=torch.uint8)
+    vals = codes.view(torch.float8_e4m3fn).float().tolist()
+    for c, v in zip(codes.tolist(), vals):
+        got = orc.e4m3_encode(v, lib=lib)
+        assert got == c, (hex(c), v, hex(got))
+
+
+def check_e4m3_encode_vs_torch(lib, n=200_000, seed=5):
+    """Against torch's float8_e4m3fn cast (round to nearest even) on
+    log-uniform magnitudes across the whole range, clamped to +-448 as the
+    quantiser saturates, and on every exact midpoint between adjacent codes."""
+    g = torch.Generator().manual_seed(seed)
+    mag = torch.exp2(torch.rand(n, generator=g) * 22.0 - 13.0)   # 2^-13 .. 2^9
+    sign = torch.where(torch.rand(n, generator=g) < 0.5, -1.0, 1.0)
+    x = (mag * sign).float()
+    pos = torch.arange(0, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).double()
+    mids = ((pos[:-1] + pos[1:]) / 2).float()                     # exact in fp32
+    x = torch.cat([x, mids, -mids, torch.tensor([0.0, -0.0, 448.0, -448.0, 1e30, -1e30])])
+    ref = x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8).tolist()
+    enc = lib.oracle_e4m3_encode
+    got = [enc(float(v)) for v in x.tolist()]
+    bad = [(v, r, g_) for v, r, g_ in zip(x.tolist(), ref, got) if r != g_]
+    assert not bad, bad[:5]
+
+
+def check_append(lib, kv_dtype, seed=3):
+    """New rows land at page_table[b][pos // P], slot pos % P for pos =
+    kv_lens[b] + t (numpy indexing, independent of the oracle's loops), with
+    bf16 bits copied / e4m3 codes from torch's cast of the fp32 quotient;
+    every other slot is unchanged."""
+    g = torch.Generator().manual_seed(seed)
+    B, T, Hkv, D, P, max_pages, num_pages = 3, 5, 2, 16, 8, 6, 30
+    kv_lens = np.array([0, 7, 22], dtype=np.int32)
+    page_table = torch.randperm(num_pages, generator=g)[:B * max_pages].reshape(B, max_pages)
+    page_table = page_table.to(torch.int32).numpy()
+    k_new = torch.randn((B, T, Hkv, D), generator=g).to(torch.bfloat16)
+    v_new = torch.randn((B, T, Hkv, D), generator=g).to(torch.bfloat16)
+    fp8 = kv_dtype == W.KV_FP8_E4M3
+    dt = np.uint8 if fp8 else np.uint16
+    k_pages = np.random.default_rng(seed).integers(0, 255, (num_pages, Hkv, P, D)).astype(dt)
+    v_pages = np.random.default_rng(seed + 1).integers(0, 255, (num_pages, Hkv, P, D)).astype(dt)
+    scale = 0.0123
+    kp, vp = orc.paged_kv_append(W.to_bits(k_new), W.to_bits(v_new), page_table, kv_lens,
+                                 k_pages, v_pages, page_size=P, kv_dtype=kv_dtype,
+                                 kv_scale=scale, lib=lib)
+
+    def coded(x):
+        if not fp8:
+            return W.to_bits(x)
+        y = (x.float() / scale).clamp(-448.0, 448.0)
+        return y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    ek, ev = k_pages.copy(), v_pages.copy()
+    for b in range(B):
+        pos = kv_lens[b] + np.arange(T)
+        pages = page_table[b, pos // P]
+        ek[pages, :, pos % P, :] = coded(k_new[b])
+        ev[pages, :, pos % P, :] = coded(v_new[b])
+    assert np.array_equal(kp, ek) and np.array_equal(vp, ev)

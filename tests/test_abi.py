@@ -184,3 +184,22 @@ def test_plan_kernel(lib):
     assert B.plan_kernel(headline_params(num_q_heads=128)) == B.PDA_KERNEL_SPLIT_FMA  # 16 rows
     assert B.plan_kernel(headline_params(head_dim=64)) == B.PDA_KERNEL_SPLIT_FMA
     assert B.plan_kernel(headline_params(head_dim=96)) == -1
+
+
+def test_append_validation(lib):
+    """paged_kv_append rejects bad params and pointers on the host."""
+    def call(**over):
+        kw = dict(batch=2, num_new=1, num_kv_heads=2, head_dim=128, page_size=16,
+                  max_pages_per_seq=4, num_pages=8, kv_dtype=B.PDA_KV_BF16, kv_scale=1.0)
+        kw.update(over)
+        p = B.PdaAppendParams(**kw)
+        ptr = 1 << 20  # never dereferenced: every case returns before device work
+        return lib.paged_kv_append(ptr, ptr, ptr, ptr, ctypes.byref(p), ptr, ptr, None)
+    assert call(num_new=0) == 1 and call(num_new=65) == 1 and call(num_kv_heads=0) == 1
+    assert call(kv_dtype=7) == 1 and call(kv_dtype=B.PDA_KV_FP8_E4M3, kv_scale=0.0) == 1
+    assert call(head_dim=96) == 2 and call(page_size=12) == 2 and call(page_size=4) == 2
+    assert call(batch=0) == 0
+    assert lib.paged_kv_append(None, None, None, None, None, None, None, None) == 1
+    p = B.PdaAppendParams(2, 1, 2, 128, 16, 4, 8, B.PDA_KV_BF16, 1.0)
+    assert lib.paged_kv_append((1 << 20) + 8, 1 << 20, 1 << 20, 1 << 20, ctypes.byref(p),
+                               1 << 20, 1 << 20, None) == 3

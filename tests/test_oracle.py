@@ -131,6 +131,9 @@ MUTATIONS = {
     "merge_weight": ("const double w = exp(ls - total);", "const double w = exp(ls - m);"),
     "bottom_right_shift": ("return kv_len - (int64_t)q_len + i;", "return kv_len - (int64_t)q_len + i - 1;"),
     "kv_scale_dropped": ("* kv_scale;\n}", ";\n}"),
+    "e4m3_ties_to_odd": ("(c & 1) == 0 && (best & 1) == 1", "(c & 1) == 1 && (best & 1) == 0"),
+    "append_slot_shifted": ("+ pos % page_size) * D;", "+ (pos + 1) % page_size) * D;"),
+    "append_scale_inverted": ("oracle_e4m3_encode(kx / kv_scale)", "oracle_e4m3_encode(kx * kv_scale)"),
 }
 
 
@@ -160,3 +163,16 @@ def test_multithreaded_oracle_is_bit_identical(lib, wl):
     ref = pins.run_oracle(inp, lib)
     got = pins.run_oracle(inp, lib, threads=4)
     assert np.array_equal(ref[0], got[0]) and np.array_equal(ref[1], got[1])
+
+
+def test_e4m3_encode_inverts_decode(lib):
+    pins.check_e4m3_encode_roundtrip(lib)
+
+
+def test_e4m3_encode_matches_torch_cast(lib):
+    pins.check_e4m3_encode_vs_torch(lib)
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3])
+def test_append_places_rows_by_page_table(lib, kv_dtype):
+    pins.check_append(lib, kv_dtype)
