@@ -55,7 +55,7 @@ extern "C" {
 /* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
 typedef struct CUstream_st* pda_stream_t;
 
-#define PDA_ABI_VERSION 1
+#define PDA_ABI_VERSION 2
 
 typedef enum {
   PDA_KV_BF16 = 0,      /* K/V elements are bfloat16 */
@@ -106,6 +106,11 @@ typedef struct {
   void* workspace;          /* device scratch (any contents), or NULL */
   size_t workspace_bytes;   /* size of workspace */
   int32_t* num_splits_out;  /* optional host out: split count used */
+  const float* sinks;       /* optional device float [Hq]: attention-sink logit of each
+                               query head (natural log, on the scale of scale*q.k):
+                               exp(sinks[h]) joins the softmax denominator and adds
+                               no value; a row with no visible key then gets
+                               out = 0, lse = sinks[h]. NULL: no sink. */
 } pda_params;
 
 /*

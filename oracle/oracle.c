@@ -33,6 +33,11 @@
  *  R5 KV pool layout is [num_pages, Hkv, page_size, D].
  *  R6 FP8 value = decode_e4m3(byte) * kv_scale, one scale for K and V.
  *  R8 a row that sees no key has out = 0 and lse = -inf.
+ *  R18 the attention-sink bias of query head h is a logit sink[h] (natural
+ *      log units, same scale as scale * q.k) that adds exp(sink[h]) to the
+ *      softmax denominator and contributes no value: out = sum_j
+ *      exp(s_j - lse) v_j with lse = ln(sum_j exp(s_j) + exp(sink[h])); a row
+ *      that sees no key has out = 0 and lse = sink[h].
  *
  * Pins (tests/test_oracle.py): brute-force dense attention over the unpaged
  * K/V, page-permutation invariance, split-merge invariance, closed forms
@@ -132,14 +137,17 @@ static int check_args(const int32_t* kv_lens, int B, int q_len, int Hq, int Hkv,
 /*
  * One output row: out[b, i, h, :] and lse[b, i, h], restricted to keys in
  * [tok_lo, tok_hi) (tok_hi < 0 means no restriction). `s` is scratch for
- * kv_lens[b] scores.
+ * kv_lens[b] scores. `sink` (natural-log units, -inf for none) is the row's
+ * attention-sink logit: one more exp(sink) term in the softmax denominator
+ * with no value vector (reading R18).
  */
 static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_pages,
                       const int32_t* page_table, const int32_t* kv_lens, int q_len,
                       int Hq, int Hkv, int D, int page_size, int max_pages,
                       int num_pages, float scale, int causal_offset, int window,
                       int kv_dtype, float kv_scale, int64_t tok_lo, int64_t tok_hi,
-                      int b, int i, int h, double* s, double* out, double* lse) {
+                      double sink, int b, int i, int h, double* s, double* out,
+                      double* lse) {
   const int G = Hq / Hkv;
   const int causal = causal_offset != ORACLE_CAUSAL_OFF;
   const double dscale = (double)scale;
@@ -174,16 +182,18 @@ static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_page
     ++nvis;
   }
 
-  if (nvis == 0) { /* reading R8 */
+  if (nvis == 0) { /* reading R8; with a sink the denominator is exp(sink) alone */
     for (int d = 0; d < D; ++d) orow[d] = 0.0;
-    *lrow = -INFINITY;
+    *lrow = sink;
     return ORACLE_OK;
   }
 
-  /* lse = m + ln sum_j exp(s_j - m)  (reading R1) */
+  /* lse = m + ln (sum_j exp(s_j - m) + exp(sink - m))  (readings R1, R18) */
+  if (sink > m) m = sink;
   double sum = 0.0;
   for (int64_t j = 0; j < L; ++j)
     if (s[j] != -INFINITY) sum += exp(s[j] - m);
+  if (sink != -INFINITY) sum += exp(sink - m);
   const double row_lse = m + log(sum);
   *lrow = row_lse;
 
@@ -209,6 +219,7 @@ static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_page
  * q          bf16 bits  [B, q_len, Hq, D]
  * k/v_pages  bf16 bits or e4m3 bytes  [num_pages, Hkv, page_size, D]
  * page_table int32 [B, max_pages]; kv_lens int32 [B]
+ * sinks      float [Hq] attention-sink logits, or NULL for none
  * out        double [B, q_len, Hq, D]; lse double [B, q_len, Hq]
  */
 int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
@@ -217,8 +228,8 @@ int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
                              int Hkv, int D, int page_size, int max_pages,
                              int num_pages, float scale, int causal_offset,
                              int window, int kv_dtype, float kv_scale,
-                             int64_t tok_lo, int64_t tok_hi, double* out,
-                             double* lse) {
+                             const float* sinks, int64_t tok_lo, int64_t tok_hi,
+                             double* out, double* lse) {
   int64_t max_len;
   int st = check_args(kv_lens, B, q_len, Hq, Hkv, D, page_size, max_pages, num_pages,
                       causal_offset, kv_dtype, &max_len);
@@ -230,7 +241,8 @@ int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
       for (int h = 0; h < Hq; ++h) {
         st = oracle_row(q, k_pages, v_pages, page_table, kv_lens, q_len, Hq, Hkv, D,
                         page_size, max_pages, num_pages, scale, causal_offset, window,
-                        kv_dtype, kv_scale, tok_lo, tok_hi, b, i, h, s, out, lse);
+                        kv_dtype, kv_scale, tok_lo, tok_hi,
+                        sinks ? (double)sinks[h] : -INFINITY, b, i, h, s, out, lse);
         if (st != ORACLE_OK) {
           free(s);
           return st;
@@ -252,7 +264,8 @@ int oracle_paged_decode_attn_mt(const uint16_t* q, const void* k_pages,
                                 int Hkv, int D, int page_size, int max_pages,
                                 int num_pages, float scale, int causal_offset,
                                 int window, int kv_dtype, float kv_scale,
-                                double* out, double* lse, int threads) {
+                                const float* sinks, double* out, double* lse,
+                                int threads) {
   int64_t max_len;
   int st = check_args(kv_lens, B, q_len, Hq, Hkv, D, page_size, max_pages, num_pages,
                       causal_offset, kv_dtype, &max_len);
@@ -272,7 +285,8 @@ int oracle_paged_decode_attn_mt(const uint16_t* q, const void* k_pages,
       const int b = (int)(r / ((int64_t)Hq * q_len));
       local = oracle_row(q, k_pages, v_pages, page_table, kv_lens, q_len, Hq, Hkv, D,
                          page_size, max_pages, num_pages, scale, causal_offset, window,
-                         kv_dtype, kv_scale, 0, -1, b, i, h, s, out, lse);
+                         kv_dtype, kv_scale, 0, -1, sinks ? (double)sinks[h] : -INFINITY,
+                         b, i, h, s, out, lse);
     }
 #pragma omp critical
     if (local != ORACLE_OK) status = local;

@@ -72,6 +72,7 @@ def _declare(lib):
         p, p, p, p, p,                      # q, k, v, page_table, kv_lens
         i32, i32, i32, i32, i32, i32, i32, i32,  # B Lq Hq Hkv D P max_pages num_pages
         ctypes.c_float, i32, i32, i32, ctypes.c_float,  # scale causal window dtype kv_scale
+        p,                                  # sinks (float [Hq]) or NULL
         ctypes.c_int64, ctypes.c_int64,     # tok_lo, tok_hi
         p, p,                               # out, lse
     ]
@@ -80,6 +81,7 @@ def _declare(lib):
         p, p, p, p, p,
         i32, i32, i32, i32, i32, i32, i32, i32,
         ctypes.c_float, i32, i32, i32, ctypes.c_float,
+        p,                                  # sinks or NULL
         p, p, i32,                          # out, lse, threads
     ]
     lib.oracle_max_threads.restype = i32
@@ -113,7 +115,7 @@ def e4m3_to_double(code: int, lib=None) -> float:
 def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
                       num_kv_heads, page_size, scale, causal_offset=CAUSAL_OFF,
                       window=0, kv_dtype=ORACLE_KV_BF16, kv_scale=1.0,
-                      tok_range=None, threads=1, lib=None):
+                      tok_range=None, threads=1, sinks=None, lib=None):
     """Run the oracle on host arrays.
 
     q_bits      uint16 [B, q_len, Hq, D]   (bf16 bit patterns)
@@ -122,6 +124,7 @@ def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
     tok_range   optional (lo, hi): keep only keys with lo <= j < hi
     threads     > 1: the same rows on that many OpenMP threads (bit-identical
                 results; no tok_range)
+    sinks       optional float [Hq]: attention-sink logit per query head
     Returns (out float64 [B, q_len, Hq, D], lse float64 [B, q_len, Hq]).
     """
     lib = lib or load()
@@ -139,6 +142,10 @@ def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
     out = np.zeros((B, q_len, Hq, D), dtype=np.float64)
     lse = np.zeros((B, q_len, Hq), dtype=np.float64)
     lo, hi = (0, -1) if tok_range is None else tok_range
+    sk = None if sinks is None else np.ascontiguousarray(sinks, dtype=np.float32)
+    if sk is not None:
+        assert sk.shape == (Hq,), sk.shape
+    skp = None if sk is None else _ptr(sk)
     if threads > 1:
         if tok_range is not None:
             raise ValueError("tok_range is only supported single-threaded")
@@ -146,7 +153,7 @@ def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
             _ptr(q_bits), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
             _ptr(kv_lens), B, q_len, Hq, num_kv_heads, D, page_size, max_pages,
             num_pages, float(scale), int(causal_offset), int(window),
-            int(kv_dtype), float(kv_scale), _ptr(out), _ptr(lse), int(threads))
+            int(kv_dtype), float(kv_scale), skp, _ptr(out), _ptr(lse), int(threads))
         if rc != 0:
             raise ValueError(f"oracle_paged_decode_attn_mt failed with status {rc}")
         return out, lse
@@ -154,7 +161,7 @@ def paged_decode_attn(q_bits, k_pages, v_pages, page_table, kv_lens, *,
         _ptr(q_bits), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
         _ptr(kv_lens), B, q_len, Hq, num_kv_heads, D, page_size, max_pages,
         num_pages, float(scale), int(causal_offset), int(window),
-        int(kv_dtype), float(kv_scale), int(lo), int(hi), _ptr(out), _ptr(lse))
+        int(kv_dtype), float(kv_scale), skp, int(lo), int(hi), _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError(f"oracle_paged_decode_attn failed with status {rc}")
     return out, lse

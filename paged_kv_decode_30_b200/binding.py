@@ -89,6 +89,7 @@ class PdaParams(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
         ("num_splits_out", ctypes.POINTER(ctypes.c_int32)),
+        ("sinks", ctypes.c_void_p),
     ]
 
 
@@ -192,11 +193,12 @@ def _stream_handle(stream) -> Optional[int]:
 def paged_decode_attn(q, k_pages, v_pages, page_table, kv_lens, *, num_kv_heads,
                       scale, causal_offset=PDA_CAUSAL_OFF, window=0, kv_scale=1.0,
                       max_kv_len=0, num_splits=0, flags=0, out=None, lse=None,
-                      workspace=None, stream=None, with_lse=True):
+                      workspace=None, stream=None, with_lse=True, sinks=None):
     """Run the library on CUDA tensors; returns (out, lse, num_splits_used).
 
     q [B, q_len, Hq, D] bf16; k/v_pages [num_pages, Hkv, P, D] bf16 or uint8
-    (e4m3 codes); page_table int32 [B, max_pages]; kv_lens int32 [B].
+    (e4m3 codes); page_table int32 [B, max_pages]; kv_lens int32 [B];
+    sinks: optional float32 CUDA tensor [Hq] of attention-sink logits.
     ``workspace``: a CUDA uint8 tensor (any contents; reusable across calls),
     or None to let the binding allocate exactly what the call needs.
     """
@@ -226,6 +228,10 @@ def paged_decode_attn(q, k_pages, v_pages, page_table, kv_lens, *, num_kv_heads,
     if workspace is not None:
         params.workspace = workspace.data_ptr()
         params.workspace_bytes = workspace.numel() * workspace.element_size()
+    if sinks is not None:
+        if not (sinks.is_cuda and sinks.dtype == torch.float32 and sinks.numel() == Hq):
+            raise ValueError("sinks must be a float32 CUDA tensor of num_q_heads entries")
+        params.sinks = sinks.data_ptr()
     used = ctypes.c_int32(0)
     params.num_splits_out = ctypes.pointer(used)
     st = lib.paged_decode_attn(

@@ -9,6 +9,8 @@
 // stored normalised with its own lse):
 //   lse = m + ln sum_s exp(lse_s - m),  m = max_s lse_s
 //   out = sum_s exp(lse_s - lse) * o_s
+// An attention-sink logit of the row's query head (optional) is one more
+// part with lse = sink and o = 0: it adds to the denominator only.
 // One warp per row, head_dim across the lanes in 8/16/32-byte vectors. Parts
 // with lse = -inf are skipped without reading their o. Launched with
 // programmatic dependent launch after the split kernel, so its CTAs are
@@ -23,14 +25,15 @@ template <int D>
 __global__ void __launch_bounds__(256) merge_states_kernel(
     const float* __restrict__ o_parts, const float* __restrict__ lse_parts,
     int num_splits, long long rows, float* __restrict__ out,
-    float* __restrict__ lse) {
+    float* __restrict__ lse, const float* __restrict__ sinks, int Hq) {
   pdl_wait_primary();  // no-op unless launched as a programmatic dependent
   constexpr int PER = D / 32;
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (row >= rows) return;
 
-  float m = -INFINITY;
+  const float sink = sinks != nullptr ? __ldg(sinks + row % Hq) : -INFINITY;
+  float m = sink;
   for (int s = 0; s < num_splits; ++s) m = fmaxf(m, __ldg(lse_parts + s * rows + row));
   float acc[PER];
 #pragma unroll
@@ -42,6 +45,7 @@ __global__ void __launch_bounds__(256) merge_states_kernel(
       const float ls = __ldg(lse_parts + s * rows + row);
       if (ls != -INFINITY) sum += expf(ls - m);
     }
+    if (sink != -INFINITY) sum += expf(sink - m);
     total = m + logf(sum);
     for (int s = 0; s < num_splits; ++s) {
       const float ls = __ldg(lse_parts + s * rows + row);
@@ -65,6 +69,6 @@ __global__ void __launch_bounds__(256) merge_states_kernel(
 
 cudaError_t launch_merge(int D, const float* o_parts, const float* lse_parts,
                          int num_splits, long long rows, float* out, float* lse,
-                         cudaStream_t stream, bool pdl);
+                         const float* sinks, int Hq, cudaStream_t stream, bool pdl);
 
 }  // namespace pda

@@ -213,7 +213,7 @@ int* device_error_word() {
 
 cudaError_t launch_merge(int D, const float* o_parts, const float* lse_parts,
                          int num_splits, long long rows, float* out, float* lse,
-                         cudaStream_t stream, bool pdl) {
+                         const float* sinks, int Hq, cudaStream_t stream, bool pdl) {
   if (rows <= 0) return cudaSuccess;
   constexpr int kWarpsPerBlock = 8;
   cudaLaunchConfig_t cfg{};
@@ -227,9 +227,9 @@ cudaError_t launch_merge(int D, const float* o_parts, const float* lse_parts,
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   switch (D) {
-    case 64: return cudaLaunchKernelEx(&cfg, merge_states_kernel<64>, o_parts, lse_parts, num_splits, rows, out, lse);
-    case 128: return cudaLaunchKernelEx(&cfg, merge_states_kernel<128>, o_parts, lse_parts, num_splits, rows, out, lse);
-    case 256: return cudaLaunchKernelEx(&cfg, merge_states_kernel<256>, o_parts, lse_parts, num_splits, rows, out, lse);
+    case 64: return cudaLaunchKernelEx(&cfg, merge_states_kernel<64>, o_parts, lse_parts, num_splits, rows, out, lse, sinks, Hq);
+    case 128: return cudaLaunchKernelEx(&cfg, merge_states_kernel<128>, o_parts, lse_parts, num_splits, rows, out, lse, sinks, Hq);
+    case 256: return cudaLaunchKernelEx(&cfg, merge_states_kernel<256>, o_parts, lse_parts, num_splits, rows, out, lse, sinks, Hq);
     default: return cudaErrorNotSupported;
   }
 }
@@ -289,7 +289,8 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   }
   if (!q || !k_pages || !v_pages || !page_table || !kv_lens || !out) return PDA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
-      !aligned(page_table, 4) || !aligned(kv_lens, 4) || (lse && !aligned(lse, 4)))
+      !aligned(page_table, 4) || !aligned(kv_lens, 4) || (lse && !aligned(lse, 4)) ||
+      (p.sinks && !aligned(p.sinks, 4)))
     return PDA_ERR_MISALIGNED;
   if (p.workspace && !aligned(p.workspace, 256)) return PDA_ERR_MISALIGNED;
 
@@ -322,6 +323,7 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   a.num_pages = p.num_pages;
   a.tile_shift = pl.tc ? 0 : ilog2(p.page_size / pl.tw);
   a.num_splits = splits;
+  a.sinks = p.sinks;
   a.row_tiles = pl.row_tiles;
   a.causal_offset = p.causal_offset;
   a.window = p.window;
@@ -389,8 +391,8 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   if (e == cudaErrorNotSupported) return PDA_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return PDA_ERR_CUDA;
   if (splits > 1 && !(pl.tc && a.fused_merge)) {
-    e = launch_merge(p.head_dim, a.o_part, a.lse_part, splits, pl.rows, out, lse, stream,
-                     (p.flags & PDA_FLAG_NO_PDL) == 0);
+    e = launch_merge(p.head_dim, a.o_part, a.lse_part, splits, pl.rows, out, lse, p.sinks,
+                     p.num_q_heads, stream, (p.flags & PDA_FLAG_NO_PDL) == 0);
     if (e != cudaSuccess) return PDA_ERR_CUDA;
   }
   if (p.num_splits_out) *p.num_splits_out = splits;
@@ -407,6 +409,7 @@ pda_status pda_merge_states(const float* o_parts, const float* lse_parts, int32_
   if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) || (lse && !aligned(lse, 4)))
     return PDA_ERR_MISALIGNED;
   const cudaError_t e = launch_merge(head_dim, o_parts, lse_parts, num_splits, rows, out, lse,
+                                     nullptr, 1,
                                      reinterpret_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? PDA_OK : PDA_ERR_CUDA;
 }

@@ -75,6 +75,7 @@ struct SplitArgs {
   int* sched;                // [0] next work item
   int* merge_ctr;            // [B * Hkv * row_tiles] splits finished per group
   int num_items;             // B * Hkv * num_splits * row_tiles
+  const float* sinks;        // [Hq] attention-sink logit per query head, or null
   int fused_merge;           // 1: the last split of a group merges it in-kernel
 };
 
@@ -525,15 +526,26 @@ __global__ void __launch_bounds__(NW * 32, 1)
         o.x += wt * x.x; o.y += wt * x.y; o.z += wt * x.z; o.w += wt * x.w;
       }
     }
+    const int i = R / a.G, h = kvh * a.G + R % a.G;
+    // attention sink of head h (one split only; with splits the merge adds
+    // it): one more exp2(sink) term in the denominator, no value
+    const float sink = a.num_splits == 1 && a.sinks ? __ldg(a.sinks + h) : -INFINITY;
     float res_lse = -INFINITY;
     if (lt > 0.f) {
-      const float inv = a.v_scale / lt;
+      float mref = mstar, l2 = lt, scl = 1.f;
+      if (sink != -INFINITY) {
+        const float sl = sink * 1.4426950408889634f;
+        mref = fmaxf(mstar, sl);
+        scl = fast_exp2(mstar - mref);
+        l2 = fmaf(lt, scl, fast_exp2(sl - mref));
+      }
+      const float inv = a.v_scale * scl / l2;
       o.x *= inv; o.y *= inv; o.z *= inv; o.w *= inv;
-      res_lse = (mstar + log2f(lt)) * 0.69314718055994531f;
+      res_lse = (mref + log2f(l2)) * 0.69314718055994531f;
     } else {
       o = make_float4(0.f, 0.f, 0.f, 0.f);
+      res_lse = sink;  // no visible key: the sink alone (-inf without one)
     }
-    const int i = R / a.G, h = kvh * a.G + R % a.G;
     const long long row = (long long)(b * a.Lq + i) * a.Hq + h;
     if (a.num_splits == 1) {
       *reinterpret_cast<float4*>(a.out + row * D + d) = o;

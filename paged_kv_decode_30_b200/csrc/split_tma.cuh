@@ -942,10 +942,26 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
       if (sid < NT) {
         const float lt = lred[sid] + lred[32 + sid] + lred[64 + sid] + lred[96 + sid];
         const bool live = lt > 0.f && !failed;
-        sm_inv[sid] = live ? a.v_scale / lt : 0.f;
         const long long row = rows[sid];
+        // attention sink of the row's head (one split only; with splits the
+        // merge adds it): one more exp2(sink) term in the denominator
+        const float sink =
+            a.num_splits == 1 && a.sinks && row >= 0 ? __ldg(a.sinks + row % a.Hq) : -INFINITY;
+        float inv = 0.f, res = failed ? -INFINITY : sink;
+        if (live) {
+          const float m = -sm_csm[sid].y;
+          float mref = m, l2 = lt, scl = 1.f;
+          if (sink != -INFINITY) {
+            const float sl = sink * kLog2e;
+            mref = fmaxf(m, sl);
+            scl = fast_exp2(m - mref);
+            l2 = fmaf(lt, scl, fast_exp2(sl - mref));
+          }
+          inv = a.v_scale * scl / l2;
+          res = (mref + log2f(l2)) * kLn2;
+        }
+        sm_inv[sid] = inv;
         if (row >= 0) {
-          const float res = live ? (log2f(lt) - sm_csm[sid].y) * kLn2 : -INFINITY;
           if (a.num_splits == 1) {
             if (a.lse) a.lse[row] = res;
           } else {
@@ -994,14 +1010,20 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
           }
 #pragma unroll
           for (int k = 0; k < RW; ++k) {
+            // the row's attention sink is one more part: lse = sink, o = 0
+            const int rr = w8 + NW8 * k;
+            const long long rrow = rr < NT ? rows[rr] : -1;
+            const float sink = a.sinks && rrow >= 0 ? __ldg(a.sinks + rrow % a.Hq) : -INFINITY;
             float m = fmaxf(fmaxf(v[k][0], v[k][1]), fmaxf(v[k][2], v[k][3]));
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+            m = fmaxf(m, sink);
             float sum = 0.f;
             if (m != -INFINITY) {
 #pragma unroll
               for (int c = 0; c < 4; ++c)
                 if (v[k][c] != -INFINITY) sum += fast_exp2((v[k][c] - m) * kLog2e);
+              if (lane == 0 && sink != -INFINITY) sum += fast_exp2((sink - m) * kLog2e);
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);

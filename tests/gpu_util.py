@@ -37,7 +37,7 @@ def run_cuda(inp, **kw):
     return out.double().cpu().numpy(), lse.double().cpu().numpy(), used
 
 
-def run_oracle(inp, seqs=None):
+def run_oracle(inp, seqs=None, sinks=None):
     """The oracle on all sequences, or on the listed ones only (their pages
     are gathered into a small pool first). Returns out, lse for those rows."""
     wl = inp["workload"]
@@ -64,7 +64,7 @@ def run_oracle(inp, seqs=None):
         W.to_bits(q), W.to_bits(kp), W.to_bits(vp), np.asarray(table, dtype=np.int32),
         np.asarray(kv, dtype=np.int32), num_kv_heads=wl.num_kv_heads,
         page_size=wl.page_size, scale=W.scale_of(wl), causal_offset=wl.causal_offset,
-        window=wl.window, kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"])
+        window=wl.window, kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"], sinks=sinks)
 
 
 def max_err(got, ref):

@@ -115,8 +115,10 @@ def visibility_matrix(L, q_len, causal_offset, window):
     return vis
 
 
-def bruteforce(inp):
-    """Textbook dense softmax attention over the unpaged K/V copies."""
+def bruteforce(inp, sinks=None):
+    """Textbook dense softmax attention over the unpaged K/V copies. An
+    attention sink enters as one more key with score sinks[h] and a zero
+    value vector."""
     wl = inp["workload"]
     B, Lq, Hq, D = inp["q"].shape
     G = wl.group
@@ -131,13 +133,17 @@ def bruteforce(inp):
         vis = visibility_matrix(L, Lq, wl.causal_offset, wl.window)
         for i in range(Lq):
             sel = vis[i]
-            if not sel.any():
-                continue
             for h in range(Hq):
                 g = h // G
                 s = scale * (K[g][sel] @ q[b, i, h])
+                Vs = V[g][sel]
+                if sinks is not None:
+                    s = np.append(s, float(sinks[h]))
+                    Vs = np.vstack([Vs, np.zeros((1, D))])
+                if s.size == 0 or np.all(np.isneginf(s)):
+                    continue
                 lse[b, i, h] = logsumexp(s)
-                out[b, i, h] = np.exp(s - lse[b, i, h]) @ V[g][sel]
+                out[b, i, h] = np.exp(s - lse[b, i, h]) @ Vs
     return out, lse
 
 
@@ -333,6 +339,8 @@ def run_all(lib):
     check_e4m3_encode_vs_torch(lib, n=20_000)
     check_append(lib, W.KV_BF16)
     check_append(lib, W.KV_FP8_E4M3)
+    for wl in (SMALL_CASES[2], SMALL_CASES[6], SMALL_CASES[7]):
+        check_sink_bruteforce(wl, lib)
 
 
 # ---------------------------------------------------------------------------
@@ -399,3 +407,33 @@ def check_append(lib, kv_dtype, seed=3):
         ek[pages, :, pos % P, :] = coded(k_new[b])
         ev[pages, :, pos % P, :] = coded(v_new[b])
     assert np.array_equal(kp, ek) and np.array_equal(vp, ev)
+
+
+# ---------------------------------------------------------------------------
+# attention sink
+
+def sink_logits(wl, seed=21):
+    """Per-query-head sink logits on the scale of the scores, one of them far
+    above every score (the sink takes almost all the weight) and one -inf."""
+    g = torch.Generator().manual_seed(seed)
+    sk = (torch.randn(wl.num_q_heads, generator=g) * 2.0).to(torch.float32)
+    sk[0] = 30.0
+    if wl.num_q_heads > 1:
+        sk[-1] = float("-inf")
+    return sk.numpy()
+
+
+def check_sink_bruteforce(wl, lib, tol=1e-12):
+    inp = W.generate(wl, device="cpu")
+    sk = sink_logits(wl)
+    ref_out, ref_lse = bruteforce(inp, sinks=sk)
+    out, lse = run_oracle(inp, lib, sinks=sk)
+    assert_close(out, ref_out, tol, f"{wl.name} sink out")
+    assert_close(lse, ref_lse, tol, f"{wl.name} sink lse")
+
+
+def check_sink_neg_inf_is_no_sink(wl, lib):
+    inp = W.generate(wl, device="cpu")
+    a_out, a_lse = run_oracle(inp, lib)
+    b_out, b_lse = run_oracle(inp, lib, sinks=np.full(wl.num_q_heads, -np.inf, np.float32))
+    assert np.array_equal(a_out, b_out) and np.array_equal(a_lse, b_lse)

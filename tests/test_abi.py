@@ -52,7 +52,7 @@ def test_only_c_abi_symbols_are_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.pda_abi_version() == 1
+    assert lib.pda_abi_version() == 2
     for code in range(8):
         assert B.status_string(code)
     assert B.status_string(99) == "unknown status"

@@ -134,6 +134,8 @@ MUTATIONS = {
     "e4m3_ties_to_odd": ("(c & 1) == 0 && (best & 1) == 1", "(c & 1) == 1 && (best & 1) == 0"),
     "append_slot_shifted": ("+ pos % page_size) * D;", "+ (pos + 1) % page_size) * D;"),
     "append_scale_inverted": ("oracle_e4m3_encode(kx / kv_scale)", "oracle_e4m3_encode(kx * kv_scale)"),
+    "sink_dropped": ("if (sink != -INFINITY) sum += exp(sink - m);", ""),
+    "sink_empty_row": ("*lrow = sink;", "*lrow = -INFINITY;"),
 }
 
 
@@ -176,3 +178,12 @@ def test_e4m3_encode_matches_torch_cast(lib):
 @pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3])
 def test_append_places_rows_by_page_table(lib, kv_dtype):
     pins.check_append(lib, kv_dtype)
+
+
+@pytest.mark.parametrize("wl", [pins.SMALL_CASES[i] for i in (0, 2, 3, 6, 7, 8)], ids=lambda w: w.name)
+def test_sink_matches_bruteforce_with_a_zero_value_key(lib, wl):
+    pins.check_sink_bruteforce(wl, lib)
+
+
+def test_sink_of_minus_infinity_changes_nothing(lib):
+    pins.check_sink_neg_inf_is_no_sink(pins.SMALL_CASES[3], lib)

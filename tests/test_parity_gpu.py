@@ -292,3 +292,28 @@ def test_cuda_graph_replays(lib):
         assert B.last_device_error() == 0
         U.assert_parity(out.double().cpu().numpy(), lse.double().cpu().numpy(), ref_out, ref_lse,
                         case.kv_dtype, f"graph replay {rep}")
+
+
+SINK_CASES = [c for c in CASES if c.head_dim == 128][:3] + \
+    [c for c in CASES if c.name.startswith("tc_fp8")][:2] + [CASES[0]]
+
+
+@pytest.mark.parametrize("case", SINK_CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("splits", [0, 1, 3])
+@pytest.mark.parametrize("kernel", ["auto", "cuda_cores", "tensor_cores_fused_merge"])
+def test_parity_attention_sink(lib, case, splits, kernel):
+    """Per-head attention-sink logits (one dominating, one -inf): the sink
+    joins the denominator in the single-split epilogue, the merge kernel or
+    the in-kernel merge."""
+    if kernel != "auto" and case.head_dim != 128:
+        pytest.skip("forced kernels apply to head_dim 128")
+    flags = {"auto": 0, "cuda_cores": B.PDA_FLAG_CUDA_CORES,
+             "tensor_cores_fused_merge": B.PDA_FLAG_TENSOR_CORES | B.PDA_FLAG_FUSED_MERGE}[kernel]
+    inp = W.generate(case)
+    g = torch.Generator().manual_seed(77)
+    sk = torch.randn(case.num_q_heads, generator=g) * 2.0
+    sk[0] = 12.0
+    sk[-1] = float("-inf")
+    ref_out, ref_lse = U.run_oracle(inp, sinks=sk.numpy())
+    out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=flags, sinks=sk.cuda())
+    U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, f"{case.name}/{kernel}/s={splits}/sink")
