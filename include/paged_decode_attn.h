@@ -214,12 +214,18 @@ PDA_API int32_t pda_choose_num_splits(const pda_params* params, int32_t num_sms)
  * o_parts    device fp32 [num_splits, rows, head_dim]
  * lse_parts  device fp32 [num_splits, rows]
  * out        device fp32 [rows, head_dim];  lse device fp32 [rows] or NULL
+ * sinks      optional device fp32 [num_q_heads]: attention-sink logit of
+ *            row r's head r % num_q_heads, one more part with lse = sink and
+ *            o = 0 (rows laid out [..., num_q_heads]); NULL for none.
  * head_dim in {64, 128, 256}; num_splits >= 1; o_parts and out 16-byte
- * aligned, lse_parts and lse 4-byte aligned.
+ * aligned, lse_parts, lse and sinks 4-byte aligned. This is also the
+ * combine step of decode context parallel: the parts are the per-GPU states
+ * of disjoint key shards.
  */
 PDA_API pda_status pda_merge_states(const float* o_parts, const float* lse_parts,
                             int32_t num_splits, int64_t rows, int32_t head_dim,
-                            float* out, float* lse, pda_stream_t stream);
+                            float* out, float* lse, const float* sinks,
+                            int32_t num_q_heads, pda_stream_t stream);
 
 /* Parameters of paged_kv_append. */
 typedef struct {

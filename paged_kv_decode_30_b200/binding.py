@@ -118,7 +118,7 @@ def load(path: Optional[str] = None):
     lib.pda_choose_num_splits.restype = i32
     lib.pda_choose_num_splits.argtypes = [pp, i32]
     lib.pda_merge_states.restype = i32
-    lib.pda_merge_states.argtypes = [vp, vp, i32, i64, i32, vp, vp, vp]
+    lib.pda_merge_states.argtypes = [vp, vp, i32, i64, i32, vp, vp, vp, i32, vp]
     lib.pda_status_string.restype = ctypes.c_char_p
     lib.pda_status_string.argtypes = [i32]
     lib.pda_last_device_error.restype = i32
@@ -293,8 +293,9 @@ def paged_kv_append(k_new, v_new, page_table, kv_lens, k_pages, v_pages, *, kv_s
         raise PdaError(st, "paged_kv_append")
 
 
-def merge_states(o_parts, lse_parts, *, out=None, lse=None, stream=None):
-    """LSE merge: o_parts [S, rows, D] fp32, lse_parts [S, rows] fp32."""
+def merge_states(o_parts, lse_parts, *, out=None, lse=None, sinks=None, stream=None):
+    """LSE merge: o_parts [S, rows, D] fp32, lse_parts [S, rows] fp32; sinks
+    optional fp32 [Hq] (row r uses sinks[r % Hq])."""
     import torch
     S, rows, D = o_parts.shape
     if out is None:
@@ -302,7 +303,8 @@ def merge_states(o_parts, lse_parts, *, out=None, lse=None, stream=None):
     if lse is None:
         lse = torch.empty((rows,), dtype=torch.float32, device=o_parts.device)
     st = load().pda_merge_states(_ptr(o_parts), _ptr(lse_parts), S, rows, D,
-                                 _ptr(out), _ptr(lse), _stream_handle(stream))
+                                 _ptr(out), _ptr(lse), _ptr(sinks),
+                                 0 if sinks is None else sinks.numel(), _stream_handle(stream))
     if st != 0:
         raise PdaError(st, "pda_merge_states")
     return out, lse

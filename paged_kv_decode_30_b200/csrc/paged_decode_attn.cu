@@ -401,15 +401,17 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
 
 pda_status pda_merge_states(const float* o_parts, const float* lse_parts, int32_t num_splits,
                             int64_t rows, int32_t head_dim, float* out, float* lse,
-                            pda_stream_t stream) {
+                            const float* sinks, int32_t num_q_heads, pda_stream_t stream) {
   if (num_splits < 1 || rows < 0) return PDA_ERR_INVALID_ARG;
+  if (sinks && num_q_heads < 1) return PDA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PDA_ERR_UNSUPPORTED;
   if (rows == 0) return PDA_OK;
   if (!o_parts || !lse_parts || !out) return PDA_ERR_INVALID_ARG;
-  if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) || (lse && !aligned(lse, 4)))
+  if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) ||
+      (lse && !aligned(lse, 4)) || (sinks && !aligned(sinks, 4)))
     return PDA_ERR_MISALIGNED;
   const cudaError_t e = launch_merge(head_dim, o_parts, lse_parts, num_splits, rows, out, lse,
-                                     nullptr, 1,
+                                     sinks, sinks ? num_q_heads : 1,
                                      reinterpret_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? PDA_OK : PDA_ERR_CUDA;
 }

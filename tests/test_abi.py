@@ -120,11 +120,11 @@ def test_empty_batch_is_a_no_op(lib):
 
 
 def test_merge_states_validation(lib):
-    st = lib.pda_merge_states(None, None, 0, 4, 128, None, None, None)
+    st = lib.pda_merge_states(None, None, 0, 4, 128, None, None, None, 0, None)
     assert st == 1
-    st = lib.pda_merge_states(None, None, 2, 4, 96, None, None, None)
+    st = lib.pda_merge_states(None, None, 2, 4, 96, None, None, None, 0, None)
     assert st == 2
-    st = lib.pda_merge_states(None, None, 2, 0, 128, None, None, None)
+    st = lib.pda_merge_states(None, None, 2, 0, 128, None, None, None, 0, None)
     assert st == 0
 
 
