@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fused-merge", action="store_true",
                     help="tensor-core kernel: merge splits in the kernel (no merge launch)")
+    ap.add_argument("--native-fp8-qk", action="store_true",
+                    help="FP8 K/V: q enters QK^T as one e4m3 term (changes the result)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the read-only HBM probe and the CUDA-graph replay (profiling runs)")
     return ap.parse_args(argv)
@@ -343,6 +345,8 @@ def run_ours(args, rank, world, local):
              "cuda_cores": B.PDA_FLAG_CUDA_CORES}[args.kernel]
     if args.fused_merge:
         flags |= B.PDA_FLAG_FUSED_MERGE
+    if args.native_fp8_qk:
+        flags |= B.PDA_FLAG_NATIVE_FP8_QK
     kw = dict(num_kv_heads=wl.num_kv_heads, scale=scale, causal_offset=wl.causal_offset,
               window=wl.window, kv_scale=inp["kv_scale"], max_kv_len=max_len,
               num_splits=args.splits, flags=flags)

@@ -84,6 +84,13 @@ typedef enum {
 #define PDA_FLAG_FUSED_MERGE 8u  /* tensor-core kernel with splits: the split that
                                     finishes last for a group of rows merges them
                                     in the kernel (no merge launch) */
+#define PDA_FLAG_NATIVE_FP8_QK 16u /* FP8 K/V on the tensor-core kernel: q enters
+                                    QK^T as one e4m3 value per element, e4m3 of
+                                    q * 2^e (nearest even; 2^e the power of two
+                                    that puts max|q| of its row in [128, 256)),
+                                    instead of an exact two-term split. Changes
+                                    the result: equal to attention with q
+                                    replaced by e4m3(q * 2^e) * 2^-e. */
 
 typedef struct {
   int32_t batch;            /* B >= 0 */

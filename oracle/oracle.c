@@ -332,6 +332,36 @@ uint8_t oracle_e4m3_encode(float x) {
 }
 
 /*
+ * Q as "native FP8 QK" uses it: each row of D bf16 values becomes
+ * e4m3(q * 2^e) * 2^-e with 2^e the power of two that puts max|q| of the row
+ * in [128, 256) (e = 7 - floor(log2 max|q|)); an all-zero row stays zero.
+ * The product q * 2^e is exact in single precision, so the quantised code is
+ * decided as the kernel decides it. The result is exactly representable in
+ * bf16 (3 mantissa bits), so it is returned as bf16 bits and the attention
+ * routine runs on it unchanged.
+ */
+int oracle_quantize_q_e4m3(const uint16_t* q, int64_t rows, int D, uint16_t* q_out) {
+  if (rows < 0 || D < 1) return ORACLE_BAD_ARG;
+  for (int64_t r = 0; r < rows; ++r) {
+    double mx = 0.0;
+    for (int d = 0; d < D; ++d) {
+      const double v = fabs(oracle_bf16_to_double(q[r * D + d]));
+      if (v > mx) mx = v;
+    }
+    const int e = mx > 0.0 ? 7 - ilogb(mx) : 0;
+    for (int d = 0; d < D; ++d) {
+      const float x = (float)ldexp(oracle_bf16_to_double(q[r * D + d]), e);
+      const double v = ldexp(oracle_e4m3_to_double(oracle_e4m3_encode(x)), -e);
+      const float f = (float)v;  /* exact */
+      uint32_t bits;
+      memcpy(&bits, &f, sizeof bits);
+      q_out[r * D + d] = (uint16_t)(bits >> 16);  /* low half is zero */
+    }
+  }
+  return ORACLE_OK;
+}
+
+/*
  * Paged KV append (the KV-cache producer): new row t of sequence b goes to
  * logical position pos = kv_lens[b] + t, i.e. page page_table[b][pos / P],
  * slot pos % P, for every kv head. bf16 pools receive the bits unchanged;

@@ -88,6 +88,8 @@ def _declare(lib):
     lib.oracle_max_threads.argtypes = []
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_quantize_q_e4m3.restype = i32
+    lib.oracle_quantize_q_e4m3.argtypes = [p, ctypes.c_int64, i32, p]
     lib.oracle_paged_kv_append.restype = i32
     lib.oracle_paged_kv_append.argtypes = [
         p, p, p, p,                          # k_new, v_new, page_table, kv_lens
@@ -194,6 +196,18 @@ def paged_kv_append(k_new_bits, v_new_bits, page_table, kv_lens, k_pages, v_page
     if rc != 0:
         raise ValueError(f"oracle_paged_kv_append failed with status {rc}")
     return kp, vp
+
+
+def quantize_q_e4m3(q_bits, lib=None):
+    """q (bf16 bits [..., D]) as native FP8 QK uses it, as bf16 bits."""
+    lib = lib or load()
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    out = np.empty_like(q_bits)
+    D = q_bits.shape[-1]
+    rc = lib.oracle_quantize_q_e4m3(_ptr(q_bits), q_bits.size // D, D, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_q_e4m3 failed with status {rc}")
+    return out
 
 
 def max_threads(lib=None) -> int:

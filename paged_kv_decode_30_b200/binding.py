@@ -23,6 +23,7 @@ PDA_FLAG_NO_PDL = 1
 PDA_FLAG_TENSOR_CORES = 2
 PDA_FLAG_CUDA_CORES = 4
 PDA_FLAG_FUSED_MERGE = 8
+PDA_FLAG_NATIVE_FP8_QK = 16
 # Size of the library's fixed partials array used by paged_decode_attn_no_alloc.
 PDA_NO_ALLOC_WORKSPACE_BYTES = 16 * 1024 * 1024
 

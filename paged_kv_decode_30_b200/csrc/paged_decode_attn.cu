@@ -378,7 +378,8 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
     a.num_items = (int)items;
     a.fused_merge = (p.flags & PDA_FLAG_FUSED_MERGE) != 0;
     const int grid = (int)std::min<long long>(items, dev->num_sms);
-    e = launch_split_tma(kv, pl.mt, k_pages, v_pages, a, grid, stream);
+    e = launch_split_tma(kv, pl.mt, fp8 && (p.flags & PDA_FLAG_NATIVE_FP8_QK) != 0, k_pages,
+                         v_pages, a, grid, stream);
   } else {
     const dim3 grid((unsigned)pl.row_tiles, (unsigned)(splits * p.num_kv_heads), (unsigned)p.batch);
     switch (p.head_dim) {

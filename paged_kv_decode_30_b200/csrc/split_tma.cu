@@ -45,11 +45,11 @@ bool make_pool_map(CUtensorMap* map, const void* base, long long rows, int elt, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KV, int NT>
+template <int KV, int NT, bool QN = false>
 cudaError_t launch_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const SplitArgs& a,
                        int grid, cudaStream_t stream) {
-  using C = TmaCfg<KV, NT>;
-  auto kern = split_tma_kernel<KV, NT>;
+  using C = TmaCfg<KV, NT, QN>;
+  auto kern = split_tma_kernel<KV, NT, QN>;
   static unsigned long long attr_set = 0;  // bit d: opt-in set on device d (< 64)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -66,8 +66,9 @@ cudaError_t launch_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const Split
 
 }  // namespace
 
-cudaError_t launch_split_tma(int kv, int nt, const void* k_pages, const void* v_pages,
-                             const SplitArgs& a, int grid, cudaStream_t stream) {
+cudaError_t launch_split_tma(int kv, int nt, bool native_qk, const void* k_pages,
+                             const void* v_pages, const SplitArgs& a, int grid,
+                             cudaStream_t stream) {
   const long long rows = (long long)a.num_pages * a.Hkv * a.page_size;
   const int elt = kv == 0 ? 2 : 1;
   const int box_rows = a.page_size < 128 ? a.page_size : 128;
@@ -79,6 +80,13 @@ cudaError_t launch_split_tma(int kv, int nt, const void* k_pages, const void* v_
     switch (nt) {
       case 4: return launch_cfg<0, 4>(mk, mv, a, grid, stream);
       case 8: return launch_cfg<0, 8>(mk, mv, a, grid, stream);
+      default: return cudaErrorNotSupported;
+    }
+  }
+  if (native_qk) {
+    switch (nt) {
+      case 16: return launch_cfg<1, 16, true>(mk, mv, a, grid, stream);
+      case 32: return launch_cfg<1, 32, true>(mk, mv, a, grid, stream);
       default: return cudaErrorNotSupported;
     }
   }

@@ -61,13 +61,17 @@ struct ItemDesc {
   int pids[PA][16];        // page ids of the item's first PA tiles (segment = page)
 };
 
-template <int KV, int NT>
+// QN (FP8 only): "native FP8 QK", Q enters the MMA as one e4m3 term per
+// element (q * 2^e rounded to nearest even, per-row power-of-two 2^e)
+// instead of the exact two-term split, so S^T has NT columns, not 2 NT.
+template <int KV, int NT, bool QN = false>
 struct TmaCfg {
   static constexpr bool BF16 = KV == 0;
+  static constexpr bool QN_ = QN;
   static constexpr int D = 128;
   static constexpr int TILE = 128;
   static constexpr int ELT = BF16 ? 2 : 1;
-  static constexpr int N1 = BF16 ? 16 : 2 * NT;  // S^T columns
+  static constexpr int N1 = BF16 ? 16 : (QN ? NT : 2 * NT);  // S^T columns
   static constexpr int N2 = BF16 ? 16 : NT;      // O^T columns
   static constexpr int STAGES = 3;
   static constexpr int KT = TILE * D * ELT;      // bytes of one K (or V) tile
@@ -132,6 +136,7 @@ struct TmaCfg {
   static constexpr int TMEM_COLS = 2 * N1 + 2 * N2 <= 64 ? 64 : (2 * N1 + 2 * N2 <= 128 ? 128 : 256);
   static constexpr int COL_S = 0, COL_O = 2 * N1;
   static_assert(BF16 ? (NT == 4 || NT == 8) : (NT == 16 || NT == 32), "rows per CTA");
+  static_assert(!(BF16 && QN), "native QK is an FP8 option");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
   static_assert(OFF_VC % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
   static_assert(sizeof(Desc) % 16 == 0 && OFF_DESC % 16 == 0 && OFF_SLOTS % 16 == 0, "alignment");
@@ -212,11 +217,11 @@ __device__ __forceinline__ void decode_item(const SplitArgs& a, int t, int& b, i
   b = u / a.Hkv;
 }
 
-template <int KV, int NT>
-__global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
+template <int KV, int NT, bool QN = false>
+__global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     split_tma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const SplitArgs a) {
-  using C = TmaCfg<KV, NT>;
+  using C = TmaCfg<KV, NT, QN>;
   using Desc = typename C::Desc;
   constexpr int PA = C::PID_AHEAD;
   constexpr unsigned FULL = 0xFFFFFFFFu;
@@ -430,7 +435,8 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
       } else if (lane < NT) {
         // Lane n: row n (hi) and row NT + n (lo) in e4m3, 128 bytes each,
         // SW128 K-major. q * 2^e2 = hi + lo / 16 exactly, with 2^e2 the power
-        // of two that puts max|q| of the row in [128, 256).
+        // of two that puts max|q| of the row in [128, 256). Native QK keeps
+        // hi alone (q quantised to e4m3 at that scale).
         const int n = lane, R = R0 + n;
         const bool live = R < a.M;
         const uint4* src = reinterpret_cast<const uint4*>(a.q);
@@ -477,8 +483,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
           }
           *reinterpret_cast<uint4*>(qbuf + (rh >> 3) * 1024 + (rh & 7) * 128 +
                                     ((c ^ (rh & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(qbuf + (rl >> 3) * 1024 + (rl & 7) * 128 +
-                                    ((c ^ (rl & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          if constexpr (!C::QN_)
+            *reinterpret_cast<uint4*>(qbuf + (rl >> 3) * 1024 + (rl & 7) * 128 +
+                                      ((c ^ (rl & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
       }
       fence_proxy_async_smem();  // the Q operand is read by the tensor core
@@ -797,6 +804,12 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
             tmem_ld16_raw(ta, sraw);
 #pragma unroll
             for (int r = 0; r < RH; ++r) s[r] = sraw[r];
+          } else if constexpr (C::QN_) {  // S = S_hi (columns r)
+            if constexpr (RH == 16) {
+              tmem_ld16_raw(ta + r0, s);
+            } else {
+              tmem_ld8(ta + r0, s);
+            }
           } else {
             float lo[RH];  // S = S_hi + S_lo / 16 (columns r and NT + r)
             if constexpr (RH == 16) {
@@ -1127,9 +1140,11 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT>::THREADS, 1)
   }
 }
 
-// Host launcher (split_tma.cu). kv: 0 bf16, 1 e4m3; nt: rows per CTA; grid:
-// persistent CTAs (at most one per SM).
-cudaError_t launch_split_tma(int kv, int nt, const void* k_pages, const void* v_pages,
-                             const SplitArgs& a, int grid, cudaStream_t stream);
+// Host launcher (split_tma.cu). kv: 0 bf16, 1 e4m3; nt: rows per CTA;
+// native_qk: FP8 with one-term e4m3 Q; grid: persistent CTAs (at most one
+// per SM).
+cudaError_t launch_split_tma(int kv, int nt, bool native_qk, const void* k_pages,
+                             const void* v_pages, const SplitArgs& a, int grid,
+                             cudaStream_t stream);
 
 }  // namespace pda

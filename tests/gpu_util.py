@@ -37,7 +37,7 @@ def run_cuda(inp, **kw):
     return out.double().cpu().numpy(), lse.double().cpu().numpy(), used
 
 
-def run_oracle(inp, seqs=None, sinks=None):
+def run_oracle(inp, seqs=None, sinks=None, native_qk=False):
     """The oracle on all sequences, or on the listed ones only (their pages
     are gathered into a small pool first). Returns out, lse for those rows."""
     wl = inp["workload"]
@@ -60,8 +60,11 @@ def run_oracle(inp, seqs=None, sinks=None):
         kp, vp = inp["k_pages"][idx], inp["v_pages"][idx]
         q = inp["q"][torch.tensor(seqs, device=inp["q"].device)]
         kv = lens[seqs]
+    qbits = W.to_bits(q)
+    if native_qk:  # the oracle mirrors the Q quantisation of native FP8 QK
+        qbits = orc.quantize_q_e4m3(qbits)
     return orc.paged_decode_attn(
-        W.to_bits(q), W.to_bits(kp), W.to_bits(vp), np.asarray(table, dtype=np.int32),
+        qbits, W.to_bits(kp), W.to_bits(vp), np.asarray(table, dtype=np.int32),
         np.asarray(kv, dtype=np.int32), num_kv_heads=wl.num_kv_heads,
         page_size=wl.page_size, scale=W.scale_of(wl), causal_offset=wl.causal_offset,
         window=wl.window, kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"], sinks=sinks)

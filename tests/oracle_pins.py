@@ -20,6 +20,10 @@ What pins what:
   * e4m3 encode: inverts torch's decode on every finite code; equals torch's
     float8_e4m3fn cast (round to nearest even) on 200k log-uniform values and
     on every exact midpoint between adjacent codes.
+  * quantize_q (native FP8 QK): equals torch's float8 cast of q * 2^e per
+    row, with 2^e from torch.frexp of the row's max |q|.
+  * sink: brute-force dense attention with the sink as one more key of zero
+    value; a -inf sink is bit-identical to none.
   * append: new rows land where numpy indexing of the page table says
     (page_table[b][pos // P], slot pos % P), as torch-cast codes for FP8;
     every other slot is unchanged.
@@ -341,6 +345,7 @@ def run_all(lib):
     check_append(lib, W.KV_FP8_E4M3)
     for wl in (SMALL_CASES[2], SMALL_CASES[6], SMALL_CASES[7]):
         check_sink_bruteforce(wl, lib)
+    check_quantize_q_vs_torch(lib)
 
 
 # ---------------------------------------------------------------------------
@@ -437,3 +442,23 @@ def check_sink_neg_inf_is_no_sink(wl, lib):
     a_out, a_lse = run_oracle(inp, lib)
     b_out, b_lse = run_oracle(inp, lib, sinks=np.full(wl.num_q_heads, -np.inf, np.float32))
     assert np.array_equal(a_out, b_out) and np.array_equal(a_lse, b_lse)
+
+
+# ---------------------------------------------------------------------------
+# native FP8 QK: the per-row e4m3 quantisation of q
+
+def check_quantize_q_vs_torch(lib, seed=8):
+    """Against torch: per row, 2^e = 2^(8 - frexp exponent of max|q|) puts
+    max|q| in [128, 256); q * 2^e through torch's float8_e4m3fn cast, back
+    times 2^-e, as bf16 bits. Rows of mixed magnitude, and a zero row."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((37, 64), generator=g) * torch.exp2(torch.randint(-12, 12, (37, 1), generator=g).float())
+    q[5] = 0.0
+    qb = q.to(torch.bfloat16)
+    mx = qb.float().abs().amax(dim=1, keepdim=True)
+    _, ex = torch.frexp(torch.where(mx > 0, mx, torch.ones_like(mx)))
+    e = torch.where(mx > 0, 8 - ex, torch.zeros_like(ex)).float()
+    ref = (qb.float() * torch.exp2(e)).clamp(-448, 448).to(torch.float8_e4m3fn).float() * torch.exp2(-e)
+    ref_bits = W.to_bits(ref.to(torch.bfloat16))
+    got = orc.quantize_q_e4m3(W.to_bits(qb), lib=lib)
+    assert np.array_equal(got, ref_bits)

@@ -136,6 +136,8 @@ MUTATIONS = {
     "append_scale_inverted": ("oracle_e4m3_encode(kx / kv_scale)", "oracle_e4m3_encode(kx * kv_scale)"),
     "sink_dropped": ("if (sink != -INFINITY) sum += exp(sink - m);", ""),
     "sink_empty_row": ("*lrow = sink;", "*lrow = -INFINITY;"),
+    "quantize_q_scale_off_by_one": ("const int e = mx > 0.0 ? 7 - ilogb(mx) : 0;",
+                                    "const int e = mx > 0.0 ? 8 - ilogb(mx) : 0;"),
 }
 
 
@@ -187,3 +189,7 @@ def test_sink_matches_bruteforce_with_a_zero_value_key(lib, wl):
 
 def test_sink_of_minus_infinity_changes_nothing(lib):
     pins.check_sink_neg_inf_is_no_sink(pins.SMALL_CASES[3], lib)
+
+
+def test_native_qk_quantisation_matches_torch(lib):
+    pins.check_quantize_q_vs_torch(lib)

@@ -317,3 +317,27 @@ def test_parity_attention_sink(lib, case, splits, kernel):
     ref_out, ref_lse = U.run_oracle(inp, sinks=sk.numpy())
     out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=flags, sinks=sk.cuda())
     U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, f"{case.name}/{kernel}/s={splits}/sink")
+
+
+NATIVE_CASES = [c for c in CASES if c.kv_dtype == FP8 and c.head_dim == 128]
+
+
+@pytest.mark.parametrize("case", NATIVE_CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_parity_native_fp8_qk(lib, case, splits):
+    """Native FP8 QK (q as one e4m3 term per element) against the oracle run
+    on the same per-row quantisation of q."""
+    inp = W.generate(case)
+    ref_out, ref_lse = U.run_oracle(inp, native_qk=True)
+    flags = B.PDA_FLAG_TENSOR_CORES | B.PDA_FLAG_NATIVE_FP8_QK
+    out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=flags)
+    U.assert_parity(out, lse, ref_out, ref_lse, FP8, f"{case.name}/native/s={splits}")
+
+
+def test_full_size_fp8_verify_native_qk(lib):
+    case = _full(W.FP8_VERIFY.name)
+    inp = W.generate(case, device="cuda")
+    out, lse, _ = U.run_cuda(inp, flags=B.PDA_FLAG_NATIVE_FP8_QK)
+    seqs = [0, 17, 63]
+    ref_out, ref_lse = U.run_oracle(inp, seqs=seqs, native_qk=True)
+    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, FP8, "fp8 verify native qk")
