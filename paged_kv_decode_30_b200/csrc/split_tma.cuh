@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
   uint64_t* s_full = bars + 2 * C::STAGES;     // [2] S^T in TMEM
   uint64_t* p_ready = s_full + 2;              // [2] P^T in shared memory
   uint64_t* o_full = s_full + 4;               // [2] O^T in TMEM
-  uint64_t* o_free = s_full + 6;               // [2] O^T read back
+  uint64_t* o_free = s_full + 6;               // [2] O^T region of an item read back
   uint64_t* v_ready = s_full + 8;              // [2] f16 V tile (FP8)
   uint64_t* desc_full = s_full + 10;           // [4] item descriptor published
   uint64_t* desc_free = desc_full + C::DSLOTS; // [4] item finished (descriptor reusable)
@@ -677,17 +677,19 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           }
           if (ok) umma_commit(&q_free[j & 1]);  // arrives once item j's S^T MMAs are done
         } else {
-          for (int n = 0; n < ntiles; ++n, ++g) {
+          // O^T of item j accumulates over its tiles in TMEM region j & 1;
+          // the region is free once the softmax warps read item j-2's O.
+          if (j >= 2) ok = mbar_wait(&o_free[j & 1], ((j >> 1) - 1) & 1, a.err);
+          for (int n = 0; ok && n < ntiles; ++n, ++g) {
             const int bb = g & 1;
             ok = !*abort_flag && mbar_wait(&p_ready[bb], (g >> 1) & 1, a.err);
-            if (ok && g >= 2) ok = mbar_wait(&o_free[bb], ((g - 2) >> 1) & 1, a.err);
             if constexpr (!C::BF16) {
               if (ok) ok = mbar_wait(&v_ready[bb], (g >> 1) & 1, a.err);
             }
             if (!ok) break;
             tmem_fence_after();
             const uint32_t pa = sbase + C::OFF_P + bb * C::P_BUF;
-            const uint32_t dt = tmem + C::COL_O + bb * C::N2;
+            const uint32_t dt = tmem + C::COL_O + (j & 1) * C::N2;
             if constexpr (C::BF16) {
               constexpr uint32_t idesc = umma_idesc_bf16(128, C::N2, true, true);
               const uint32_t va = sbase + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT;
@@ -695,7 +697,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
               for (int s = 0; s < C::TILE / 16; ++s)
                 umma_f16(dt, umma_desc(va + s * 2048, C::HALF, 1024, kSw128),
                          umma_desc(pa + s * 2 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE),
-                         idesc, s > 0);
+                         idesc, n > 0 || s > 0);
               umma_commit(&empty[g % C::STAGES]);  // K and V of the stage are consumed
             } else {
               constexpr uint32_t idesc = umma_idesc_f16(128, C::N2, true, true);
@@ -704,7 +706,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
               for (int s = 0; s < C::TILE / 16; ++s)
                 umma_f16(dt, umma_desc(va + s * 2048, C::HALF, 1024, kSw128),
                          umma_desc(pa + s * 2 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE),
-                         idesc, s > 0);
+                         idesc, n > 0 || s > 0);
             }
             umma_commit(&o_full[bb]);
             issued = g + 1;
@@ -755,38 +757,28 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       float2* sm_csm = reinterpret_cast<float2*>(sl + C::SL_CSM);
       float* sm_thr = reinterpret_cast<float*>(sl + C::SL_THR);
       float* sm_mraw = reinterpret_cast<float*>(sl + C::SL_MRAW);
-      uint32_t resc = 0;  // bit (tile & 1): that tile moved the running max
       float l_part[RH], acc[RH];
 #pragma unroll
       for (int r = 0; r < RH; ++r) {
         l_part[r] = 0.f;
         acc[r] = 0.f;
       }
-
-      auto accumulate = [&](int k) -> bool {  // fold O^T of tile k into acc
-        const int bb = k & 1;
-        const bool ok_w = __all_sync(FULL, mbar_wait(&o_full[bb], (k >> 1) & 1, a.err));
-        if (!ok_w) return false;
-        tmem_fence_after();
-        float o[C::BF16 ? 16 : RH];
-        const uint32_t ta = tmem + lane_off + C::COL_O + bb * C::N2;
-        if constexpr (C::BF16) {
-          tmem_ld16_raw(ta, o);  // rows 0..NT-1 from P_hi, NT..2NT-1 from P_lo
-        } else if constexpr (RH == 16) {
-          tmem_ld16_raw(ta + r0, o);
+      // O^T of this item accumulates in TMEM region j & 1 (columns = rows;
+      // bf16: rows NT.. hold the P_lo part). This thread's part of it:
+      const uint32_t o_tm = tmem + lane_off + C::COL_O + (j & 1) * C::N2 + (C::BF16 ? 0 : r0);
+      constexpr int OC = C::BF16 ? 16 : RH;  // TMEM columns this thread reads
+      auto load_o = [&](float* o) {
+        if constexpr (OC == 16) {
+          tmem_ld16_raw(o_tm, o);
         } else {
-          tmem_ld8(ta + r0, o);
+          tmem_ld8(o_tm, o);
         }
-        tmem_fence_before();
-        mbar_arrive(&o_free[bb]);
-        const float* al = sm_alpha + bb * 32 + r0;
-        const bool rs = (resc >> bb) & 1u;
-#pragma unroll
-        for (int r = 0; r < RH; ++r) {
-          const float ov = C::BF16 ? o[r] + o[NT + r] : o[r];  // P = P_hi + P_lo
-          acc[r] = rs ? fmaf(acc[r], al[r], ov) : acc[r] + ov;
-        }
-        return true;
+      };
+      // wait until the O^T MMAs of tile k have completed (all lanes agree)
+      auto wait_o = [&](int k) -> bool {
+        const bool ok_w = __all_sync(FULL, mbar_wait(&o_full[k & 1], (k >> 1) & 1, a.err));
+        if (ok_w) tmem_fence_after();
+        return ok_w;
       };
 
       bool acc_ok = true;
@@ -863,7 +855,6 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           acc_ok = false;
           break;
         }
-        resc = (resc & ~(1u << bb)) | ((uint32_t)flag << bb);
         if (flag) {
 #pragma unroll
           for (int r = 0; r < RH; ++r) {
@@ -885,6 +876,28 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           named_bar(2, ST);
 #pragma unroll
           for (int r = 0; r < RH; ++r) l_part[r] *= sm_alpha[bb * 32 + r0 + r];
+          // the O^T accumulated so far (tiles before this one) moves to the
+          // new max too, before this tile's P V lands on it (rare: the max
+          // moves on an item's first tile, then only on a jump of 2^8)
+          // (a failed wait only clears acc_ok: the next tile's barrier, or
+          // the item's last one, then stops every softmax warp together)
+          if (n > 0) {
+            if (wait_o(g - 1)) {
+              float o[OC];
+              load_o(o);
+              const float* al = sm_alpha + bb * 32 + r0;
+#pragma unroll
+              for (int c = 0; c < OC; ++c) o[c] *= al[C::BF16 ? (c % NT) : c];
+              if constexpr (OC == 16) {
+                tmem_st16(o_tm, o);
+              } else {
+                tmem_st8(o_tm, o);
+              }
+              tmem_fence_before();
+            } else {
+              acc_ok = false;
+            }
+          }
         }
         float* p = s;
 #pragma unroll
@@ -895,6 +908,11 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           l_part[r] += p[r];
           l_part[r + 1] += p[r + 1];
         }
+        // P^T buffer bb was last read by the O^T MMAs of tile g - 2. Waiting
+        // for them every tile also keeps this warp's o_full phases in step,
+        // so the o_full(g - 1) waits above and after the loop never see a
+        // phase that is two behind.
+        if (g >= 2 && !wait_o(g - 2)) acc_ok = false;
         // P^T row of token i (row-major over the N2 columns, swizzled chunks)
         uint8_t* sp = smem + C::OFF_P + bb * C::P_BUF + (i >> 3) * C::P_SBO + (i & 7) * C::P_ROW;
         const int pswz = C::P_ROW == 64 ? ((i & 7) >> 1) & 3 : ((i & 7) >> 2) & 1;
@@ -930,9 +948,19 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         tmem_fence_before();
         mbar_arrive(&p_ready[bb]);
         if (sid == 0) *tiles_done = g + 1;  // lets the scheduler draw more work
-        if (n >= 1) acc_ok = accumulate(g - 1);
       }
-      if (__all_sync(FULL, acc_ok && ntiles > 0 && !*abort_flag)) acc_ok = accumulate(g - 1);
+      // the item's O^T once its last tile's MMAs are done
+      if (__all_sync(FULL, acc_ok && ntiles > 0 && !*abort_flag)) {
+        acc_ok = wait_o(g - 1);
+        if (acc_ok) {
+          float o[OC];
+          load_o(o);
+#pragma unroll
+          for (int r = 0; r < RH; ++r) acc[r] = C::BF16 ? o[r] + o[NT + r] : o[r];  // P = P_hi + P_lo
+        }
+      }
+      tmem_fence_before();
+      mbar_arrive(&o_free[j & 1]);  // region j & 1 may take item j + 2
       ok = named_bar_and(2, ST, acc_ok);
       if (!ok) *abort_flag = 1;
 
