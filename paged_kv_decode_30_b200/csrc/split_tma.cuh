@@ -29,16 +29,17 @@
 //        (MN-major), B = P^T split into bf16 hi + lo rows (N = 16).
 //      FP8 K/V: S^T with kind::f8f6f4 straight from the e4m3 K stage, B =
 //        [Q_hi; Q_lo], an exact two-term e4m3 split of each bf16 q row
-//        scaled by a power of two; O^T with kind::f16 on V converted to f16
-//        by warps 8-11.
-//  * warps 3-6 (softmax): thread i = TMEM lane i = token i of S^T and
+//        scaled by a power of two; O^T with kind::f8f6f4 straight from the
+//        e4m3 V stage (MN-major), B = P^T as two e4m3 terms [P_hi; 16 P_lo].
+//  * warps 3-6 (and, FP8, 8-19 by item rows: groups of four warps with 8
+//    rows each) (softmax): thread i = TMEM lane i = token i of S^T and
 //    head-dim element i of O^T. p = exp2(s * c - m) in fp32 with a lazily
-//    moved running max; P^T to shared memory; O^T folded into fp32 registers.
+//    moved running max; P^T to shared memory. O^T accumulates in TMEM over
+//    the item's tiles; a tile that moves the max rescales it in place first.
 //    On tiles with keys that no row may see they also zero those keys' V
-//    rows in the stage (bf16), so NaN bytes never meet a zero weight in the
-//    MMA. After an item: normalise and store O and the LSE (or the split's
+//    rows in the stage, so NaN bytes never meet a zero weight in the MMA.
+//    After an item: normalise and store O and the LSE (or the split's
 //    partials; the split that arrives last for its rows merges them all).
-//  * warps 8-11 (FP8 only, converters): V stage e4m3 -> f16 operand tile.
 //  * Every wait is bounded; group exits go through bar.red.and.
 #pragma once
 
@@ -72,29 +73,29 @@ struct TmaCfg {
   static constexpr int TILE = 128;
   static constexpr int ELT = BF16 ? 2 : 1;
   static constexpr int N1 = BF16 ? 16 : (QN ? NT : 2 * NT);  // S^T columns
-  static constexpr int N2 = BF16 ? 16 : NT;      // O^T columns
-  static constexpr int STAGES = 3;
+  // O^T columns: bf16, the P_hi and P_lo rows (N = 16); FP8, P_hi then
+  // 16 * P_lo (two e4m3 terms per weight), summed as O_hi + O_lo / 16
+  static constexpr int N2 = BF16 ? 16 : 2 * NT;
+  static constexpr int STAGES = BF16 ? 3 : 5;
   static constexpr int KT = TILE * D * ELT;      // bytes of one K (or V) tile
   static constexpr int STAGE = 2 * KT;           // K then V
   static constexpr int HALF = TILE * 128;        // one 128-byte column of SW128 atoms
-  static constexpr int VC = TILE * D * 2;        // converted f16 V tile (FP8 only)
-  static constexpr int NVC = BF16 ? 0 : 2;
   static constexpr int Q_ROWS = N1;
   static constexpr int Q_BYTES = Q_ROWS * D * (BF16 ? 2 : 1);
   static constexpr int Q_HALF = (Q_ROWS / 8) * 1024;  // bf16: 64-element half of each row
   static constexpr int Q_BUF = ((Q_BYTES + 1023) / 1024) * 1024;  // one of two Q buffers
-  static constexpr int P_ROW = N2 * 2;                 // bytes per token row of P^T
+  static constexpr int P_ROW = N2 * ELT;               // bytes per token row of P^T
   static constexpr int P_SBO = 8 * P_ROW;
   static constexpr int P_BYTES = (TILE / 8) * P_SBO;
   static constexpr uint32_t P_SWIZZLE = P_ROW == 64 ? 4u : 6u;  // SW64 / SW32
-  // warp roles. FP8 items have up to 32 rows: two groups of four softmax
-  // warps (SOFT0.., SOFT1..) take half the rows each, so each thread carries
-  // 16 rows and each SM sub-partition has two softmax warps to interleave.
-  static constexpr int PROD = 0, S_MMA = 1, O_MMA = 2, SOFT0 = 3, SCHED = 7, CONV0 = 8, SOFT1 = 12;
-  static constexpr int SOFT_H = BF16 ? 1 : 2;       // row halves
+  // warp roles. FP8 items have 16 or 32 rows: SOFT_H groups of four
+  // softmax warps (warps 3-6, then 8-11, 12-15, 16-19) take 8 rows each, so
+  // each SM sub-partition interleaves SOFT_H softmax warps.
+  static constexpr int PROD = 0, S_MMA = 1, O_MMA = 2, SOFT0 = 3, SCHED = 7, SOFTX = 8;
+  static constexpr int SOFT_H = BF16 ? 1 : NT / 8;  // row groups
   static constexpr int RH = NT / SOFT_H;             // rows per softmax thread
   static constexpr int SOFT_THREADS = 128 * SOFT_H;
-  static constexpr int WARPS = BF16 ? 8 : 16;
+  static constexpr int WARPS = 8 + 4 * (SOFT_H - 1);
   static constexpr int THREADS = WARPS * 32;
   // work-queue depths
   static constexpr int DSLOTS = 4;                 // item descriptors in flight
@@ -114,11 +115,10 @@ struct TmaCfg {
   static constexpr int SLOT = SL_MRAW + 32 * 4;
   // shared memory map (1024-aligned where swizzled)
   static constexpr int OFF_STAGE = 0;
-  static constexpr int OFF_VC = OFF_STAGE + STAGES * STAGE;
-  static constexpr int OFF_Q = OFF_VC + NVC * VC;
+  static constexpr int OFF_Q = OFF_STAGE + STAGES * STAGE;
   static constexpr int OFF_P = OFF_Q + 2 * Q_BUF;
   static constexpr int P_BUF = ((P_BYTES + 1023) / 1024) * 1024;
-  static constexpr int OFF_WMAX = OFF_P + 2 * P_BUF;
+  static constexpr int OFF_WMAX = OFF_P + 2 * P_BUF;  // [4 warps][32 rows]
   static constexpr int OFF_ALPHA = OFF_WMAX + 4 * 32 * 4;
   static constexpr int OFF_LRED = OFF_ALPHA + 2 * 32 * 4;
   static constexpr int OFF_INV = OFF_LRED + 4 * 32 * 4;  // v_scale / l per row
@@ -126,9 +126,9 @@ struct TmaCfg {
   static constexpr int OFF_DESC = OFF_SLOTS + 2 * SLOT;
   static constexpr int OFF_PIDS = OFF_DESC + DSLOTS * (int)sizeof(Desc);
   static constexpr int OFF_BAR = OFF_PIDS + PID_SLOTS * 16 * 4;
-  // full[S], empty[S], s_full[2], p_ready[2], o_full[2], o_free[2], v_ready[2],
+  // full[S], empty[S], s_full[2], p_ready[2], o_full[2], o_free[2],
   // desc_full[4], desc_free[4], q_ready[2], st_free[2], q_free[2]
-  static constexpr int NUM_BARS = 2 * STAGES + 10 + 2 * DSLOTS + 6;
+  static constexpr int NUM_BARS = 2 * STAGES + 8 + 2 * DSLOTS + 6;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_FLAGS = OFF_TMEM_SLOT + 8;   // [0] abort, [1] merge flag, [2] tiles done
   static constexpr int SMEM = OFF_FLAGS + 16;
@@ -138,7 +138,8 @@ struct TmaCfg {
   static_assert(BF16 ? (NT == 4 || NT == 8) : (NT == 16 || NT == 32), "rows per CTA");
   static_assert(!(BF16 && QN), "native QK is an FP8 option");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
-  static_assert(OFF_VC % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
+  static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
+  static_assert(BF16 || RH == 8, "FP8: 8 rows per softmax thread");
   static_assert(sizeof(Desc) % 16 == 0 && OFF_DESC % 16 == 0 && OFF_SLOTS % 16 == 0, "alignment");
 };
 
@@ -146,6 +147,11 @@ struct TmaCfg {
 __host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+// kind::f8f6f4 with e4m3 A and B, fp32 D, both operands MN-major (A = V^T
+// with the head dimension contiguous, B = P^T with the rows contiguous).
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3_mn(int M, int N) {
+  return umma_idesc_e4m3(M, N) | (1u << 15) | (1u << 16);
 }
 // kind::f16 with bf16 A and B.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
@@ -194,6 +200,13 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
   return r;
 }
 
+// Two e4m3 codes (low byte first) -> two floats, exactly.
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t codes) {
+  const __half2_raw hr =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes & 0xFFFFu), __NV_E4M3);
+  return make_float2(__half2float(__ushort_as_half(hr.x)), __half2float(__ushort_as_half(hr.y)));
+}
+
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code & 0xFF), __NV_E4M3);
   return __half2float(*reinterpret_cast<const __half*>(&h));
@@ -238,8 +251,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
   uint64_t* p_ready = s_full + 2;              // [2] P^T in shared memory
   uint64_t* o_full = s_full + 4;               // [2] O^T in TMEM
   uint64_t* o_free = s_full + 6;               // [2] O^T region of an item read back
-  uint64_t* v_ready = s_full + 8;              // [2] f16 V tile (FP8)
-  uint64_t* desc_full = s_full + 10;           // [4] item descriptor published
+  uint64_t* desc_full = s_full + 8;            // [4] item descriptor published
   uint64_t* desc_free = desc_full + C::DSLOTS; // [4] item finished (descriptor reusable)
   uint64_t* q_ready = desc_free + C::DSLOTS;   // [2] Q operand + per-row state written
   uint64_t* st_free = q_ready + 2;             // [2] per-row state of an item released
@@ -254,14 +266,13 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::BF16 ? 1 : 2);
+      mbar_init(&empty[s], 1);  // the O^T MMAs of the tile are done
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_ready[i], C::SOFT_THREADS);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], C::SOFT_THREADS);
-      mbar_init(&v_ready[i], 128);
       mbar_init(&q_ready[i], 32);
       mbar_init(&st_free[i], 1);
       mbar_init(&q_free[i], 1);
@@ -670,7 +681,6 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
               for (int s = 0; s < C::D / 32; ++s)
                 umma_f8(dt, umma_desc(ka + s * 32, 16, 1024, kSw128),
                         umma_desc(qa + s * 32, 16, 1024, kSw128), idesc, s > 0);
-              umma_commit(&empty[g % C::STAGES]);  // the K half of the stage is consumed
             }
             umma_commit(&s_full[bb]);
             issued = g + 1;
@@ -683,31 +693,30 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           for (int n = 0; ok && n < ntiles; ++n, ++g) {
             const int bb = g & 1;
             ok = !*abort_flag && mbar_wait(&p_ready[bb], (g >> 1) & 1, a.err);
-            if constexpr (!C::BF16) {
-              if (ok) ok = mbar_wait(&v_ready[bb], (g >> 1) & 1, a.err);
-            }
             if (!ok) break;
             tmem_fence_after();
             const uint32_t pa = sbase + C::OFF_P + bb * C::P_BUF;
             const uint32_t dt = tmem + C::COL_O + (j & 1) * C::N2;
+            const uint32_t va = sbase + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT;
             if constexpr (C::BF16) {
               constexpr uint32_t idesc = umma_idesc_bf16(128, C::N2, true, true);
-              const uint32_t va = sbase + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT;
 #pragma unroll
               for (int s = 0; s < C::TILE / 16; ++s)
                 umma_f16(dt, umma_desc(va + s * 2048, C::HALF, 1024, kSw128),
                          umma_desc(pa + s * 2 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE),
                          idesc, n > 0 || s > 0);
-              umma_commit(&empty[g % C::STAGES]);  // K and V of the stage are consumed
             } else {
-              constexpr uint32_t idesc = umma_idesc_f16(128, C::N2, true, true);
-              const uint32_t va = sbase + C::OFF_VC + bb * C::VC;
+              // A = V^T straight from the e4m3 V stage: each token row is one
+              // 128-byte swizzle row holding all 128 head-dim elements, so the
+              // MN-major atom is 128 elements x 8 tokens; 32 tokens per MMA.
+              constexpr uint32_t idesc = umma_idesc_e4m3_mn(128, C::N2);
 #pragma unroll
-              for (int s = 0; s < C::TILE / 16; ++s)
-                umma_f16(dt, umma_desc(va + s * 2048, C::HALF, 1024, kSw128),
-                         umma_desc(pa + s * 2 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE),
-                         idesc, n > 0 || s > 0);
+              for (int s = 0; s < C::TILE / 32; ++s)
+                umma_f8(dt, umma_desc(va + s * 4096, C::HALF, 1024, kSw128),
+                        umma_desc(pa + s * 4 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE),
+                        idesc, n > 0 || s > 0);
             }
+            umma_commit(&empty[g % C::STAGES]);  // K and V of the stage are consumed
             umma_commit(&o_full[bb]);
             issued = g + 1;
           }
@@ -721,15 +730,15 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     }
     __syncwarp();
   } else if ((warp >= C::SOFT0 && warp < C::SOFT0 + 4) ||
-             (C::SOFT_H == 2 && warp >= C::SOFT1 && warp < C::SOFT1 + 4)) {
+             (C::SOFT_H > 1 && warp >= C::SOFTX && warp < C::SOFTX + 4 * (C::SOFT_H - 1))) {
     // ======================= softmax / accumulate ============================
     constexpr int RH = C::RH;
     constexpr int ST = C::SOFT_THREADS;
     const int q4 = warp & 3;
-    const int half = (C::SOFT_H == 2 && warp >= C::SOFT1) ? 1 : 0;
-    const int r0 = half * RH;        // this thread's rows: r0 .. r0 + RH - 1
+    const int grp = warp < C::SCHED ? 0 : 1 + (warp - C::SOFTX) / 4;  // row group
+    const int r0 = grp * RH;         // this thread's rows: r0 .. r0 + RH - 1
     const int i = 32 * q4 + lane;    // TMEM lane: token of S^T, element of O^T
-    const int sid = half * 128 + i;  // 0 .. ST - 1
+    const int sid = grp * 128 + i;   // 0 .. ST - 1
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     float* wmax = reinterpret_cast<float*>(smem + C::OFF_WMAX);
     float* sm_alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
@@ -763,15 +772,25 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         l_part[r] = 0.f;
         acc[r] = 0.f;
       }
-      // O^T of this item accumulates in TMEM region j & 1 (columns = rows;
-      // bf16: rows NT.. hold the P_lo part). This thread's part of it:
+      // O^T of this item accumulates in TMEM region j & 1, one column per
+      // row and weight term: bf16, columns r (P_hi) and NT + r (P_lo) of the
+      // 16; FP8, columns r (P_hi) and NT + r (16 P_lo). This thread reads its
+      // RH rows of both terms: o[0 .. RH) and o[RH .. 2 RH) (bf16: all 16).
       const uint32_t o_tm = tmem + lane_off + C::COL_O + (j & 1) * C::N2 + (C::BF16 ? 0 : r0);
-      constexpr int OC = C::BF16 ? 16 : RH;  // TMEM columns this thread reads
+      constexpr int OC = C::BF16 ? 16 : 2 * RH;
       auto load_o = [&](float* o) {
-        if constexpr (OC == 16) {
+        if constexpr (C::BF16) {
           tmem_ld16_raw(o_tm, o);
         } else {
-          tmem_ld8(o_tm, o);
+          tmem_ld8x2(o_tm, o_tm + NT, o, o + RH);
+        }
+      };
+      auto store_o = [&](const float* o) {
+        if constexpr (C::BF16) {
+          tmem_st16(o_tm, o);
+        } else {
+          tmem_st8(o_tm, o);
+          tmem_st8(o_tm + NT, o + RH);
         }
       };
       // wait until the O^T MMAs of tile k have completed (all lanes agree)
@@ -825,14 +844,12 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             const int2 lh = rng[r0 + r];
             if (!(jt >= lh.x && jt < lh.y)) s[r] = -INFINITY;
           }
-          if constexpr (C::BF16) {
-            if (jt < lo_u || jt >= hi_u) {  // zero V row i of the stage (2 halves)
-              uint8_t* vrow = smem + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT + i * 128;
+          if (jt < lo_u || jt >= hi_u) {  // zero V row i of the stage (bf16: 2 halves)
+            uint8_t* vrow = smem + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT + i * 128;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(vrow + C::HALF + c * 16) = make_uint4(0, 0, 0, 0);
-              }
+            for (int c = 0; c < 8; ++c) {
+              *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+              if constexpr (C::BF16) *reinterpret_cast<uint4*>(vrow + C::HALF + c * 16) = make_uint4(0, 0, 0, 0);
             }
           }
         }
@@ -887,12 +904,8 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
               load_o(o);
               const float* al = sm_alpha + bb * 32 + r0;
 #pragma unroll
-              for (int c = 0; c < OC; ++c) o[c] *= al[C::BF16 ? (c % NT) : c];
-              if constexpr (OC == 16) {
-                tmem_st16(o_tm, o);
-              } else {
-                tmem_st8(o_tm, o);
-              }
+              for (int c = 0; c < OC; ++c) o[c] *= al[C::BF16 ? (c % NT) : (c % RH)];
+              store_o(o);
               tmem_fence_before();
             } else {
               acc_ok = false;
@@ -933,16 +946,23 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             *reinterpret_cast<uint4*>(sp + ((0 ^ pswz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          // f16 columns r0 .. r0 + RH - 1: chunks r0/8 .. r0/8 + RH/8 - 1
+          // e4m3 bytes r0 .. r0 + 7: P_hi = e4m3(p); bytes NT + r0 ..:
+          // 16 (p - P_hi) in e4m3, so P_hi + P_lo keeps about 8 significant
+          // bits (p <= 2^8, well inside the e4m3 range)
+          uint32_t hi[2], lo[2];
 #pragma unroll
-          for (int c8 = 0; c8 < RH / 8; ++c8) {
-            uint4 w;
-            w.x = pack_f16x2(p[8 * c8 + 0], p[8 * c8 + 1]);
-            w.y = pack_f16x2(p[8 * c8 + 2], p[8 * c8 + 3]);
-            w.z = pack_f16x2(p[8 * c8 + 4], p[8 * c8 + 5]);
-            w.w = pack_f16x2(p[8 * c8 + 6], p[8 * c8 + 7]);
-            *reinterpret_cast<uint4*>(sp + (((r0 / 8 + c8) ^ pswz) << 4)) = w;
+          for (int r = 0; r < RH; r += 4) {
+            const uint32_t h01 = f32x2_to_e4m3x2(p[r], p[r + 1]);
+            const uint32_t h23 = f32x2_to_e4m3x2(p[r + 2], p[r + 3]);
+            const float2 d01 = e4m3x2_to_f32x2(h01), d23 = e4m3x2_to_f32x2(h23);
+            hi[r / 4] = h01 | (h23 << 16);
+            lo[r / 4] = f32x2_to_e4m3x2(16.f * (p[r] - d01.x), 16.f * (p[r + 1] - d01.y)) |
+                        (f32x2_to_e4m3x2(16.f * (p[r + 2] - d23.x), 16.f * (p[r + 3] - d23.y)) << 16);
           }
+          // 8-byte halves of 16-byte chunks, chunk index swizzled per row
+          const int bh = r0, bl = NT + r0;
+          *reinterpret_cast<uint2*>(sp + ((((bh >> 4) ^ pswz) << 4) | (bh & 15))) = make_uint2(hi[0], hi[1]);
+          *reinterpret_cast<uint2*>(sp + ((((bl >> 4) ^ pswz) << 4) | (bl & 15))) = make_uint2(lo[0], lo[1]);
         }
         fence_proxy_async_smem();
         tmem_fence_before();
@@ -955,8 +975,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         if (acc_ok) {
           float o[OC];
           load_o(o);
+          // bf16: P = P_hi + P_lo; FP8: P = P_hi + (16 P_lo) / 16
 #pragma unroll
-          for (int r = 0; r < RH; ++r) acc[r] = C::BF16 ? o[r] + o[NT + r] : o[r];  // P = P_hi + P_lo
+          for (int r = 0; r < RH; ++r) acc[r] = C::BF16 ? o[r] + o[NT + r] : fmaf(o[RH + r], 0.0625f, o[r]);
         }
       }
       tmem_fence_before();
@@ -1036,7 +1057,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           // w8, w8 + 4 * SOFT_H, ...; lane l holds splits l, l + 32, l + 64, l + 96.
           constexpr int NW8 = 4 * C::SOFT_H;
           constexpr int RW = (NT + NW8 - 1) / NW8;
-          const int w8 = half * 4 + q4;
+          const int w8 = grp * 4 + q4;
           float v[RW][4];
 #pragma unroll
           for (int k = 0; k < RW; ++k) {
@@ -1105,56 +1126,6 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       }
     }
     if (!ok) *abort_flag = 1;
-  } else if (warp >= C::CONV0 && warp < C::CONV0 + 4) {
-    if constexpr (!C::BF16) {
-      // ======================= V converters (FP8) ============================
-      const int t = tid - C::CONV0 * 32;  // token 0..127
-      int g = 0;
-      bool ok = true;
-      for (int j = 0; ok; ++j) {
-        ok = !*abort_flag && mbar_wait(&desc_full[j & (C::DSLOTS - 1)], (j / C::DSLOTS) & 1, a.err);
-        if (!named_bar_and(1, 128, ok)) {
-          ok = false;
-          break;
-        }
-        const Desc& d = descs[j & (C::DSLOTS - 1)];
-        if (d.b < 0) break;
-        const int kfirst = d.kfirst, ntiles = d.ntiles, lo_u = d.lo_u, hi_u = d.hi_u;
-        for (int n = 0; n < ntiles; ++n, ++g) {
-          const int st = g % C::STAGES;
-          const int bb = g & 1;
-          ok = !*abort_flag && mbar_wait(&full[st], (g / C::STAGES) & 1, a.err);
-          if (ok && g >= 2) ok = mbar_wait(&o_full[bb], ((g - 2) >> 1) & 1, a.err);
-          uint4 raw[8];
-          if (ok) {
-            const uint8_t* vrow =
-                smem + C::OFF_STAGE + st * C::STAGE + C::KT + (t >> 3) * 1024 + (t & 7) * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              raw[c] = *reinterpret_cast<const uint4*>(vrow + ((c ^ (t & 7)) << 4));
-          }
-          if (!named_bar_and(1, 128, ok)) {
-            ok = false;
-            break;
-          }
-          if (t == 0) mbar_arrive(&empty[st]);  // the V half of the stage is consumed
-          const int jt = (kfirst + n) * C::TILE + t;
-          const bool v_zero = jt < lo_u || jt >= hi_u;
-          uint8_t* dst = smem + C::OFF_VC + bb * C::VC + (t >> 3) * 1024 + (t & 7) * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {  // 16 e4m3 -> two 8-element f16 chunks
-            const int j0 = 2 * c, j1 = 2 * c + 1;
-            const uint4 f0 = v_zero ? make_uint4(0, 0, 0, 0) : e4m3x8_to_f16x8(make_uint2(raw[c].x, raw[c].y));
-            const uint4 f1 = v_zero ? make_uint4(0, 0, 0, 0) : e4m3x8_to_f16x8(make_uint2(raw[c].z, raw[c].w));
-            *reinterpret_cast<uint4*>(dst + (j0 >> 3) * C::HALF + (((j0 & 7) ^ (t & 7)) << 4)) = f0;
-            *reinterpret_cast<uint4*>(dst + (j1 >> 3) * C::HALF + (((j1 & 7) ^ (t & 7)) << 4)) = f1;
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&v_ready[bb]);
-        }
-      }
-      if (!ok) *abort_flag = 1;
-    }
   }
 
   pdl_launch_dependents();
