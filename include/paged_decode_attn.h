@@ -144,7 +144,8 @@ typedef struct {
  * scratch. It holds the split partials when the call splits the KV range,
  * and, for the tensor-core kernel (see pda_plan_kernel), a header of
  * counters: the work queue of its persistent CTAs and, per (sequence, kv
- * head, row tile), how many splits have finished (the last one merges).
+ * head, row tile) and softmax row group, how many splits have finished
+ * (the last one merges).
  * The call zeroes that header itself (one small memset on `stream` before
  * the launch), so the workspace's contents before the call do not matter
  * and a call captured in a CUDA graph replays correctly. Every partial slot

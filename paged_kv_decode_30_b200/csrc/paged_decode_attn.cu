@@ -175,7 +175,7 @@ int choose_splits(const pda_params* p, const Plan& pl, int num_sms) {
 }
 
 // Workspace layout. The tensor-core kernel keeps its work-queue counter and
-// one split-arrival counter per (sequence, kv head, row tile) at the front
+// split-arrival counters per (sequence, kv head, row tile) at the front
 // (zeroed by a memset on the call's stream before the launch); the split
 // partials follow (o_part then lse_part).
 struct WsLayout {
@@ -191,7 +191,7 @@ WsLayout ws_layout(const pda_params* p, const Plan& pl, int splits) {
   WsLayout w{};
   if (pl.tc) {
     const size_t groups = (size_t)p->batch * (size_t)p->num_kv_heads * (size_t)pl.row_tiles;
-    w.counters = round256(kMergeCtrOffset + groups * sizeof(int));
+    w.counters = round256(kMergeCtrOffset + groups * pda::kMergeCtrPerGroup * sizeof(int));
   }
   w.o_off = w.lse_off = w.total = w.counters;
   if (splits > 1) {
@@ -358,8 +358,8 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
       a.sched = reinterpret_cast<int*>(base);
       a.merge_ctr = reinterpret_cast<int*>(base + kMergeCtrOffset);
       // the counters start at zero for this call
-      const size_t used = kMergeCtrOffset +
-          (size_t)p.batch * p.num_kv_heads * pl.row_tiles * sizeof(int);
+      const size_t used = kMergeCtrOffset + (size_t)p.batch * p.num_kv_heads * pl.row_tiles *
+                                                pda::kMergeCtrPerGroup * sizeof(int);
       if (cudaMemsetAsync(base, 0, used, stream) != cudaSuccess) return PDA_ERR_CUDA;
     }
     if (splits > 1) {

@@ -50,6 +50,10 @@
 
 namespace pda {
 
+// Split-arrival counters per (sequence, kv head, row tile): one for each
+// softmax row group of the tensor-core kernel (at most four).
+constexpr int kMergeCtrPerGroup = 4;
+
 struct SplitArgs {
   const uint16_t* q;         // bf16 bits [B, Lq, Hq, D]
   const uint8_t* k_pages;    // pool bytes [num_pages, Hkv, P, D]
@@ -73,7 +77,8 @@ struct SplitArgs {
   // persistent tensor-core kernel only (counters zeroed by the host just
   // before the launch, in stream order):
   int* sched;                // [0] next work item
-  int* merge_ctr;            // [B * Hkv * row_tiles] splits finished per group
+  int* merge_ctr;            // [B * Hkv * row_tiles * kMergeCtrPerGroup] splits finished
+                             // per (group, softmax row group)
   int num_items;             // B * Hkv * num_splits * row_tiles
   const float* sinks;        // [Hq] attention-sink logit per query head, or null
   int fused_merge;           // 1: the last split of a group merges it in-kernel

@@ -73,8 +73,11 @@ struct TmaCfg {
   static constexpr int TILE = 128;
   static constexpr int ELT = BF16 ? 2 : 1;
   static constexpr int N1 = BF16 ? 16 : (QN ? NT : 2 * NT);  // S^T columns
-  // O^T columns: bf16, the P_hi and P_lo rows (N = 16); FP8, P_hi then
-  // 16 * P_lo (two e4m3 terms per weight), summed as O_hi + O_lo / 16
+  // O^T columns: bf16, the P_hi and P_lo rows (N = 16); FP8, two e4m3 terms
+  // per weight, P_hi and 16 P_lo, summed as O_hi + O_lo / 16. FP8 columns
+  // (and S^T columns with the two-term Q) go by row group: group k owns
+  // columns 16k .. 16k + 7 (hi term of rows 8k .. 8k + 7) and 16k + 8 ..
+  // 16k + 15 (lo term), so a thread reads its rows' terms in one load.
   static constexpr int N2 = BF16 ? 16 : 2 * NT;
   static constexpr int STAGES = BF16 ? 3 : 5;
   static constexpr int KT = TILE * D * ELT;      // bytes of one K (or V) tile
@@ -112,13 +115,18 @@ struct TmaCfg {
   static constexpr int SL_CSM = SL_CS + 32 * 4;       // {score scale, -m} per row
   static constexpr int SL_THR = SL_CSM + 32 * 8;      // lazy-rescale threshold per row
   static constexpr int SL_MRAW = SL_THR + 32 * 4;     // running max per row (-inf at start)
-  static constexpr int SLOT = SL_MRAW + 32 * 4;
+  static constexpr int SL_SINK = SL_MRAW + 32 * 4;    // attention-sink logit per row (-inf: none)
+  static constexpr int SLOT = SL_SINK + 32 * 4;
   // shared memory map (1024-aligned where swizzled)
   static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_Q = OFF_STAGE + STAGES * STAGE;
   static constexpr int OFF_P = OFF_Q + 2 * Q_BUF;
   static constexpr int P_BUF = ((P_BYTES + 1023) / 1024) * 1024;
-  static constexpr int OFF_WMAX = OFF_P + 2 * P_BUF;  // [4 warps][32 rows]
+  // FP8: a 32-token x 128 tile of e4m3 ones, the A operand of the MMAs that
+  // sum P^T per row into TMEM (the softmax normaliser)
+  static constexpr int ONES = BF16 ? 0 : 32 * 128;
+  static constexpr int OFF_ONES = OFF_P + 2 * P_BUF;
+  static constexpr int OFF_WMAX = OFF_ONES + ONES;  // [4 warps][32 rows]
   static constexpr int OFF_ALPHA = OFF_WMAX + 4 * 32 * 4;
   static constexpr int OFF_LRED = OFF_ALPHA + 2 * 32 * 4;
   static constexpr int OFF_INV = OFF_LRED + 4 * 32 * 4;  // v_scale / l per row
@@ -130,15 +138,18 @@ struct TmaCfg {
   // desc_full[4], desc_free[4], q_ready[2], st_free[2], q_free[2]
   static constexpr int NUM_BARS = 2 * STAGES + 8 + 2 * DSLOTS + 6;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_FLAGS = OFF_TMEM_SLOT + 8;   // [0] abort, [1] merge flag, [2] tiles done
-  static constexpr int SMEM = OFF_FLAGS + 16;
+  // [0] abort, [1] tiles done, [4 + k] merge flag of row group k
+  static constexpr int OFF_FLAGS = OFF_TMEM_SLOT + 8;
+  static constexpr int SMEM = OFF_FLAGS + 32;
   static constexpr int SMEM_ALLOC = SMEM + 1024;  // slack for the 1024-byte alignment check
-  static constexpr int TMEM_COLS = 2 * N1 + 2 * N2 <= 64 ? 64 : (2 * N1 + 2 * N2 <= 128 ? 128 : 256);
-  static constexpr int COL_S = 0, COL_O = 2 * N1;
+  // S^T and O^T regions (two each), then, FP8, two row-sum regions
+  static constexpr int COL_S = 0, COL_O = 2 * N1, COL_L = COL_O + 2 * N2;
+  static constexpr int COLS_USED = COL_L + (BF16 ? 0 : 2 * N2);
+  static constexpr int TMEM_COLS = COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
   static_assert(BF16 ? (NT == 4 || NT == 8) : (NT == 16 || NT == 32), "rows per CTA");
   static_assert(!(BF16 && QN), "native QK is an FP8 option");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
-  static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
+  static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 && OFF_ONES % 1024 == 0, "alignment");
   static_assert(BF16 || RH == 8, "FP8: 8 rows per softmax thread");
   static_assert(sizeof(Desc) % 16 == 0 && OFF_DESC % 16 == 0 && OFF_SLOTS % 16 == 0, "alignment");
 };
@@ -257,8 +268,8 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
   uint64_t* st_free = q_ready + 2;             // [2] per-row state of an item released
   uint64_t* q_free = st_free + 2;              // [2] S^T MMAs of an item done (its Q reusable)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
-  volatile int* merge_flag = abort_flag + 1;
-  volatile int* tiles_done = abort_flag + 2;  // tiles the softmax warps have finished
+  volatile int* tiles_done = abort_flag + 1;  // tiles the softmax warps have finished
+  volatile int* merge_flag = abort_flag + 4;  // [row group]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
   Desc* descs = reinterpret_cast<Desc*>(smem + C::OFF_DESC);
   auto slot_of = [&](int j) { return smem + C::OFF_SLOTS + (j & 1) * C::SLOT; };
@@ -274,15 +285,15 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], C::SOFT_THREADS);
       mbar_init(&q_ready[i], 32);
-      mbar_init(&st_free[i], 1);
+      mbar_init(&st_free[i], C::SOFT_H);  // one arrival per softmax row group
       mbar_init(&q_free[i], 1);
     }
     for (int i = 0; i < C::DSLOTS; ++i) {
       mbar_init(&desc_full[i], 32);
-      mbar_init(&desc_free[i], 1);
+      mbar_init(&desc_free[i], C::SOFT_H);
     }
     abort_flag[0] = 0;
-    merge_flag[0] = 0;
+    for (int k = 0; k < 4; ++k) merge_flag[k] = 0;
     tiles_done[0] = 0;
     fence_mbar_init();
   }
@@ -302,6 +313,10 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     if constexpr (C::BF16) {
       for (int c = i; c < 2 * C::P_BUF / 16; c += 128)
         reinterpret_cast<uint4*>(smem + C::OFF_P)[c] = make_uint4(0, 0, 0, 0);
+    } else {
+      for (int c = i; c < C::ONES / 16; c += 128)  // e4m3 1.0 = 0x38
+        reinterpret_cast<uint4*>(smem + C::OFF_ONES)[c] =
+            make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
     }
     fence_proxy_async_smem();  // read by the tensor core
   }
@@ -406,11 +421,14 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         const int R = R0 + lane;
         int lo = 0, hi = 0;
         long long row = -1;  // output row [b, qi, h] of packed row R (-1: padding)
+        float sink = -INFINITY;
         if (R < a.M) {
-          const int qi = R / a.G;
+          const int qi = R / a.G, h = kvh * a.G + (R - qi * a.G);
           row_range(a, d.L, qi, lo, hi);
-          row = (long long)(b * a.Lq + qi) * a.Hq + kvh * a.G + (R - qi * a.G);
+          row = (long long)(b * a.Lq + qi) * a.Hq + h;
+          if (a.sinks) sink = __ldg(a.sinks + h);
         }
+        reinterpret_cast<float*>(sl + C::SL_SINK)[lane] = sink;
         reinterpret_cast<long long*>(sl + C::SL_ROWS)[lane] = row;
         reinterpret_cast<int2*>(sl + C::SL_RANGE)[lane] = make_int2(lo, hi);
         reinterpret_cast<float2*>(sl + C::SL_CSM)[lane] = make_float2(1.f, 0.f);
@@ -444,7 +462,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         }
         if (lane < NT) cs[lane] = a.qk_scale_log2;
       } else if (lane < NT) {
-        // Lane n: row n (hi) and row NT + n (lo) in e4m3, 128 bytes each,
+        // Lane n: the hi and lo operand rows of item row n in e4m3, 128 bytes each,
         // SW128 K-major. q * 2^e2 = hi + lo / 16 exactly, with 2^e2 the power
         // of two that puts max|q| of the row in [128, 256). Native QK keeps
         // hi alone (q quantised to e4m3 at that scale).
@@ -468,7 +486,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         const int e2 = mx > 0.f ? 8 - ilogbf(mx) - 1 : 0;  // mx * 2^e2 < 256 <= 448
         const float sc = ldexpf(1.f, e2);
         cs[n] = ldexpf(a.qk_scale_log2, -e2);
-        const int rh = n, rl = NT + n;
+        // operand rows in row-group order: hi of row n at 16 (n / 8) + n % 8,
+        // its lo 8 rows later (native QK: hi of row n at n)
+        const int rh = C::QN_ ? n : 16 * (n >> 3) + (n & 7), rl = rh + 8;
 #pragma unroll 2
         for (int c = 0; c < 8; ++c) {  // pass 2 (L1 hits): 16 elements -> a chunk of hi and of lo
           float f[16];
@@ -687,8 +707,8 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           }
           if (ok) umma_commit(&q_free[j & 1]);  // arrives once item j's S^T MMAs are done
         } else {
-          // O^T of item j accumulates over its tiles in TMEM region j & 1;
-          // the region is free once the softmax warps read item j-2's O.
+          // O^T (FP8: and the row sums) of item j accumulate over its tiles
+          // in TMEM region j & 1, free once the softmax warps read item j-2's.
           if (j >= 2) ok = mbar_wait(&o_free[j & 1], ((j >> 1) - 1) & 1, a.err);
           for (int n = 0; ok && n < ntiles; ++n, ++g) {
             const int bb = g & 1;
@@ -715,6 +735,14 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
                 umma_f8(dt, umma_desc(va + s * 4096, C::HALF, 1024, kSw128),
                         umma_desc(pa + s * 4 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE),
                         idesc, n > 0 || s > 0);
+              // row sums of P^T (the normaliser, in every TMEM lane): the same
+              // B operand against a tile of ones
+              const uint32_t lt = tmem + C::COL_L + (j & 1) * C::N2;
+#pragma unroll
+              for (int s = 0; s < C::TILE / 32; ++s)
+                umma_f8(lt, umma_desc(sbase + C::OFF_ONES, C::HALF, 1024, kSw128),
+                        umma_desc(pa + s * 4 * C::P_SBO, C::P_BYTES, C::P_SBO, C::P_SWIZZLE),
+                        idesc, n > 0 || s > 0);
             }
             umma_commit(&empty[g % C::STAGES]);  // K and V of the stage are consumed
             umma_commit(&o_full[bb]);
@@ -731,27 +759,35 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     __syncwarp();
   } else if ((warp >= C::SOFT0 && warp < C::SOFT0 + 4) ||
              (C::SOFT_H > 1 && warp >= C::SOFTX && warp < C::SOFTX + 4 * (C::SOFT_H - 1))) {
-    // ======================= softmax / accumulate ============================
+    // ======================= softmax ==========================================
+    // A group of four warps (one per TMEM lane quarter) owns RH rows and
+    // synchronises only within itself, on named barrier 2 + group; the
+    // groups meet only through mbarriers (p_ready and o_free count every
+    // softmax thread, st_free and desc_free one arrival per group), so no
+    // group ever waits on a named barrier for another.
     constexpr int RH = C::RH;
-    constexpr int ST = C::SOFT_THREADS;
+    constexpr int GT = 128;          // threads of a group
     const int q4 = warp & 3;
     const int grp = warp < C::SCHED ? 0 : 1 + (warp - C::SOFTX) / 4;  // row group
+    const int gbar = 2 + grp;        // the group's named barrier
     const int r0 = grp * RH;         // this thread's rows: r0 .. r0 + RH - 1
     const int i = 32 * q4 + lane;    // TMEM lane: token of S^T, element of O^T
-    const int sid = grp * 128 + i;   // 0 .. ST - 1
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     float* wmax = reinterpret_cast<float*>(smem + C::OFF_WMAX);
     float* sm_alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
     float* lred = reinterpret_cast<float*>(smem + C::OFF_LRED);
-    float* sm_inv = reinterpret_cast<float*>(smem + C::OFF_INV);
+    float* sm_lse = reinterpret_cast<float*>(smem + C::OFF_INV);
     const long long rows_total = (long long)a.B * a.Lq * a.Hq;
     constexpr float kLn2 = 0.69314718055994531f, kLog2e = 1.4426950408889634f;
+    // this thread's column offset in an S^T / O^T / row-sum region
+    const uint32_t col_s = C::BF16 ? 0 : (C::QN_ ? r0 : 2 * r0);
+    const uint32_t col_o = C::BF16 ? 0 : 2 * r0;
     int g = 0;  // tiles of this CTA so far (over all items)
     bool ok = true;
     for (int j = 0; ok; ++j) {
       ok = !*abort_flag && mbar_wait(&desc_full[j & (C::DSLOTS - 1)], (j / C::DSLOTS) & 1, a.err);
       if (ok && descs[j & (C::DSLOTS - 1)].b >= 0) ok = mbar_wait(&q_ready[j & 1], (j >> 1) & 1, a.err);
-      if (!named_bar_and(2, ST, ok)) {
+      if (!named_bar_and(gbar, GT, ok)) {
         ok = false;
         break;
       }
@@ -766,33 +802,15 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       float2* sm_csm = reinterpret_cast<float2*>(sl + C::SL_CSM);
       float* sm_thr = reinterpret_cast<float*>(sl + C::SL_THR);
       float* sm_mraw = reinterpret_cast<float*>(sl + C::SL_MRAW);
-      float l_part[RH], acc[RH];
+      const float* sm_sink = reinterpret_cast<const float*>(sl + C::SL_SINK);
+      float l_part[RH];  // bf16: this thread's part of the row sums
 #pragma unroll
-      for (int r = 0; r < RH; ++r) {
-        l_part[r] = 0.f;
-        acc[r] = 0.f;
-      }
-      // O^T of this item accumulates in TMEM region j & 1, one column per
-      // row and weight term: bf16, columns r (P_hi) and NT + r (P_lo) of the
-      // 16; FP8, columns r (P_hi) and NT + r (16 P_lo). This thread reads its
-      // RH rows of both terms: o[0 .. RH) and o[RH .. 2 RH) (bf16: all 16).
-      const uint32_t o_tm = tmem + lane_off + C::COL_O + (j & 1) * C::N2 + (C::BF16 ? 0 : r0);
-      constexpr int OC = C::BF16 ? 16 : 2 * RH;
-      auto load_o = [&](float* o) {
-        if constexpr (C::BF16) {
-          tmem_ld16_raw(o_tm, o);
-        } else {
-          tmem_ld8x2(o_tm, o_tm + NT, o, o + RH);
-        }
-      };
-      auto store_o = [&](const float* o) {
-        if constexpr (C::BF16) {
-          tmem_st16(o_tm, o);
-        } else {
-          tmem_st8(o_tm, o);
-          tmem_st8(o_tm + NT, o + RH);
-        }
-      };
+      for (int r = 0; r < RH; ++r) l_part[r] = 0.f;
+      // O^T (and, FP8, the row sums) of this item accumulate in TMEM region
+      // j & 1: bf16, 16 columns (r: P_hi, NT + r: P_lo), all read by every
+      // thread; FP8, this group's 16 columns (hi terms of its rows, then lo).
+      const uint32_t o_tm = tmem + lane_off + C::COL_O + (j & 1) * C::N2 + col_o;
+      const uint32_t l_tm = tmem + lane_off + C::COL_L + (j & 1) * C::N2 + col_o;
       // wait until the O^T MMAs of tile k have completed (all lanes agree)
       auto wait_o = [&](int k) -> bool {
         const bool ok_w = __all_sync(FULL, mbar_wait(&o_full[k & 1], (k >> 1) & 1, a.err));
@@ -809,27 +827,19 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         float s[RH];  // scores (then probabilities) of this thread's rows
         if (ok_s) {
           tmem_fence_after();
-          const uint32_t ta = tmem + lane_off + C::COL_S + bb * C::N1;
+          const uint32_t ta = tmem + lane_off + C::COL_S + bb * C::N1 + col_s;
           if constexpr (C::BF16) {
             float sraw[16];
             tmem_ld16_raw(ta, sraw);
 #pragma unroll
             for (int r = 0; r < RH; ++r) s[r] = sraw[r];
-          } else if constexpr (C::QN_) {  // S = S_hi (columns r)
-            if constexpr (RH == 16) {
-              tmem_ld16_raw(ta + r0, s);
-            } else {
-              tmem_ld8(ta + r0, s);
-            }
-          } else {
-            float lo[RH];  // S = S_hi + S_lo / 16 (columns r and NT + r)
-            if constexpr (RH == 16) {
-              tmem_ld16x2(ta + r0, ta + NT + r0, s, lo);
-            } else {
-              tmem_ld8x2(ta + r0, ta + NT + r0, s, lo);
-            }
+          } else if constexpr (C::QN_) {  // S = S_hi
+            tmem_ld8(ta, s);
+          } else {  // S = S_hi + S_lo / 16 (the group's hi columns, then lo)
+            float sraw[16];
+            tmem_ld16_raw(ta, sraw);
 #pragma unroll
-            for (int r = 0; r < RH; ++r) s[r] = fmaf(lo[r], 0.0625f, s[r]);
+            for (int r = 0; r < RH; ++r) s[r] = fmaf(sraw[RH + r], 0.0625f, sraw[r]);
           }
         } else {
 #pragma unroll
@@ -844,19 +854,23 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             const int2 lh = rng[r0 + r];
             if (!(jt >= lh.x && jt < lh.y)) s[r] = -INFINITY;
           }
-          if (jt < lo_u || jt >= hi_u) {  // zero V row i of the stage (bf16: 2 halves)
+          // zero V row i of the stage (bf16: 2 halves) where no row sees key
+          // jt; group 0 only. Chunks in rotated order: the 8 rows of a
+          // 1 KB swizzle atom hit 8 different bank groups.
+          if (grp == 0 && (jt < lo_u || jt >= hi_u)) {
             uint8_t* vrow = smem + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT + i * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
-              if constexpr (C::BF16) *reinterpret_cast<uint4*>(vrow + C::HALF + c * 16) = make_uint4(0, 0, 0, 0);
+              const int cc = (c + i) & 7;
+              *reinterpret_cast<uint4*>(vrow + cc * 16) = make_uint4(0, 0, 0, 0);
+              if constexpr (C::BF16) *reinterpret_cast<uint4*>(vrow + C::HALF + cc * 16) = make_uint4(0, 0, 0, 0);
             }
           }
         }
         // Lazy rescale: the running max m of each row (log2 domain) only moves
         // when a score exceeds it by more than kRescaleLog2, so p = exp2(x - m)
-        // stays <= 2^kRescaleLog2 (well inside f16) and most tiles skip the
-        // per-tile max exchange. The test runs on raw scores against
+        // stays <= 2^kRescaleLog2 (well inside f16 and e4m3) and most tiles
+        // skip the per-tile max exchange. The test runs on raw scores against
         // thr = (m + kRescaleLog2) / cs (-inf until the row's first finite
         // score), so it is one compare per score.
         constexpr float kRescaleLog2 = 8.f;
@@ -866,8 +880,8 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           const float4 t = reinterpret_cast<const float4*>(sm_thr + r0)[r / 4];
           want = want | (s[r] > t.x) | (s[r + 1] > t.y) | (s[r + 2] > t.z) | (s[r + 3] > t.w);
         }
-        // one barrier decides for the whole tile (and propagates failures)
-        const bool flag = named_bar_or_and(2, ST, want, ok_s, &ok_s);
+        // one group barrier decides for the tile (and propagates failures)
+        const bool flag = named_bar_or_and(gbar, GT, want, ok_s, &ok_s);
         if (!ok_s) {
           acc_ok = false;
           break;
@@ -878,34 +892,43 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             const float wm = redux_max(s[r]);
             if (lane == r) wmax[q4 * 32 + r0 + r] = wm;
           }
-          named_bar(2, ST);
-          if (sid < NT) {
-            const float cs = sm_cs[sid];
-            const float st = fmaxf(fmaxf(wmax[sid], wmax[32 + sid]), fmaxf(wmax[64 + sid], wmax[96 + sid]));
-            const float m_old = sm_mraw[sid];
+          named_bar(gbar, GT);
+          if (i < RH) {
+            const int rr = r0 + i;
+            const float cs = sm_cs[rr];
+            const float st = fmaxf(fmaxf(wmax[rr], wmax[32 + rr]), fmaxf(wmax[64 + rr], wmax[96 + rr]));
+            const float m_old = sm_mraw[rr];
             const float m_new = fmaxf(m_old, st * cs);  // -inf stays -inf (cs > 0)
             const float m_use = m_new == -INFINITY ? 0.f : m_new;
-            sm_alpha[bb * 32 + sid] = m_old == -INFINITY ? 0.f : fast_exp2(m_old - m_use);
-            sm_mraw[sid] = m_new;
-            sm_csm[sid] = make_float2(cs, -m_use);
-            sm_thr[sid] = m_new == -INFINITY ? -INFINITY : (m_use + kRescaleLog2) / cs;
+            sm_alpha[bb * 32 + rr] = m_old == -INFINITY ? 0.f : fast_exp2(m_old - m_use);
+            sm_mraw[rr] = m_new;
+            sm_csm[rr] = make_float2(cs, -m_use);
+            sm_thr[rr] = m_new == -INFINITY ? -INFINITY : (m_use + kRescaleLog2) / cs;
           }
-          named_bar(2, ST);
+          named_bar(gbar, GT);
+          const float* al = sm_alpha + bb * 32 + r0;
+          if constexpr (C::BF16) {
 #pragma unroll
-          for (int r = 0; r < RH; ++r) l_part[r] *= sm_alpha[bb * 32 + r0 + r];
-          // the O^T accumulated so far (tiles before this one) moves to the
-          // new max too, before this tile's P V lands on it (rare: the max
-          // moves on an item's first tile, then only on a jump of 2^8)
-          // (a failed wait only clears acc_ok: the next tile's barrier, or
-          // the item's last one, then stops every softmax warp together)
+            for (int r = 0; r < RH; ++r) l_part[r] *= al[r];
+          }
+          // What the tiles before this one accumulated (O^T, FP8 also the row
+          // sums) moves to the new max before this tile's MMAs add to it
+          // (rare: the max moves on an item's first tile, then only on a jump
+          // of 2^8). A failed wait only clears acc_ok: the group's next
+          // barrier then stops all four of its warps together.
           if (n > 0) {
             if (wait_o(g - 1)) {
-              float o[OC];
-              load_o(o);
-              const float* al = sm_alpha + bb * 32 + r0;
+              float o[16];
+              tmem_ld16_raw(o_tm, o);
 #pragma unroll
-              for (int c = 0; c < OC; ++c) o[c] *= al[C::BF16 ? (c % NT) : (c % RH)];
-              store_o(o);
+              for (int c = 0; c < 16; ++c) o[c] *= al[C::BF16 ? (c % NT) : (c % RH)];
+              tmem_st16(o_tm, o);
+              if constexpr (!C::BF16) {
+                tmem_ld16_raw(l_tm, o);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) o[c] *= al[c % RH];
+                tmem_st16(l_tm, o);
+              }
               tmem_fence_before();
             } else {
               acc_ok = false;
@@ -918,13 +941,15 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           const float4 c = reinterpret_cast<const float4*>(sm_csm + r0)[r / 2];
           p[r] = fast_exp2(fmaf(s[r], c.x, c.y));
           p[r + 1] = fast_exp2(fmaf(s[r + 1], c.z, c.w));
-          l_part[r] += p[r];
-          l_part[r + 1] += p[r + 1];
+          if constexpr (C::BF16) {
+            l_part[r] += p[r];
+            l_part[r + 1] += p[r + 1];
+          }
         }
-        // P^T buffer bb was last read by the O^T MMAs of tile g - 2. Waiting
-        // for them every tile also keeps this warp's o_full phases in step,
-        // so the o_full(g - 1) waits above and after the loop never see a
-        // phase that is two behind.
+        // P^T buffer bb was last read by the MMAs of tile g - 2. Waiting for
+        // them every tile also keeps this warp's o_full phases in step, so
+        // the o_full(g - 1) waits above and after the loop never see a phase
+        // that is two behind.
         if (g >= 2 && !wait_o(g - 2)) acc_ok = false;
         // P^T row of token i (row-major over the N2 columns, swizzled chunks)
         uint8_t* sp = smem + C::OFF_P + bb * C::P_BUF + (i >> 3) * C::P_SBO + (i & 7) * C::P_ROW;
@@ -946,9 +971,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             *reinterpret_cast<uint4*>(sp + ((0 ^ pswz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          // e4m3 bytes r0 .. r0 + 7: P_hi = e4m3(p); bytes NT + r0 ..:
-          // 16 (p - P_hi) in e4m3, so P_hi + P_lo keeps about 8 significant
-          // bits (p <= 2^8, well inside the e4m3 range)
+          // the group's 16 columns (one 16-byte chunk): e4m3 P_hi = e4m3(p)
+          // of its 8 rows, then 16 (p - P_hi) in e4m3, so P_hi + P_lo / 16
+          // keeps about 8 significant bits (p <= 2^8, inside the e4m3 range)
           uint32_t hi[2], lo[2];
 #pragma unroll
           for (int r = 0; r < RH; r += 4) {
@@ -959,70 +984,104 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             lo[r / 4] = f32x2_to_e4m3x2(16.f * (p[r] - d01.x), 16.f * (p[r + 1] - d01.y)) |
                         (f32x2_to_e4m3x2(16.f * (p[r + 2] - d23.x), 16.f * (p[r + 3] - d23.y)) << 16);
           }
-          // 8-byte halves of 16-byte chunks, chunk index swizzled per row
-          const int bh = r0, bl = NT + r0;
-          *reinterpret_cast<uint2*>(sp + ((((bh >> 4) ^ pswz) << 4) | (bh & 15))) = make_uint2(hi[0], hi[1]);
-          *reinterpret_cast<uint2*>(sp + ((((bl >> 4) ^ pswz) << 4) | (bl & 15))) = make_uint2(lo[0], lo[1]);
+          *reinterpret_cast<uint4*>(sp + ((grp ^ pswz) << 4)) = make_uint4(hi[0], hi[1], lo[0], lo[1]);
         }
         fence_proxy_async_smem();
         tmem_fence_before();
         mbar_arrive(&p_ready[bb]);
-        if (sid == 0) *tiles_done = g + 1;  // lets the scheduler draw more work
+        if (grp == 0 && i == 0) *tiles_done = g + 1;  // lets the scheduler draw more work
       }
-      // the item's O^T once its last tile's MMAs are done
+      // the item's O^T (FP8: and row sums) once its last tile's MMAs are done
+      float acc[RH], lsum[RH];
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        acc[r] = 0.f;
+        lsum[r] = 0.f;
+      }
       if (__all_sync(FULL, acc_ok && ntiles > 0 && !*abort_flag)) {
         acc_ok = wait_o(g - 1);
         if (acc_ok) {
-          float o[OC];
-          load_o(o);
-          // bf16: P = P_hi + P_lo; FP8: P = P_hi + (16 P_lo) / 16
+          float o[16];
+          tmem_ld16_raw(o_tm, o);
+          if constexpr (C::BF16) {
 #pragma unroll
-          for (int r = 0; r < RH; ++r) acc[r] = C::BF16 ? o[r] + o[NT + r] : fmaf(o[RH + r], 0.0625f, o[r]);
+            for (int r = 0; r < RH; ++r) acc[r] = o[r] + o[NT + r];  // P = P_hi + P_lo
+          } else {
+#pragma unroll
+            for (int r = 0; r < RH; ++r) acc[r] = fmaf(o[RH + r], 0.0625f, o[r]);  // P_hi + (16 P_lo) / 16
+            tmem_ld16_raw(l_tm, o);
+#pragma unroll
+            for (int r = 0; r < RH; ++r) lsum[r] = fmaf(o[RH + r], 0.0625f, o[r]);
+          }
         }
       }
       tmem_fence_before();
       mbar_arrive(&o_free[j & 1]);  // region j & 1 may take item j + 2
-      ok = named_bar_and(2, ST, acc_ok);
+      ok = named_bar_and(gbar, GT, acc_ok);
       if (!ok) *abort_flag = 1;
 
       // ---- epilogue: normaliser and LSE per row, then the O rows ----------
+      if constexpr (C::BF16) {
+        // row sums: over the lanes, then over the group's four warps
+#pragma unroll
+        for (int r = 0; r < RH; ++r) {
+          float v = l_part[r];
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+          l_part[r] = v;
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int r = 0; r < RH; ++r) lred[q4 * 32 + r0 + r] = l_part[r];
+        }
+        named_bar(gbar, GT);
+#pragma unroll
+        for (int r = 0; r < RH; ++r)
+          lsum[r] = lred[r0 + r] + lred[32 + r0 + r] + lred[64 + r0 + r] + lred[96 + r0 + r];
+      }
+      // Every thread derives its rows' normalisers itself (the inputs are the
+      // same for all of them; an approximate division, 2 ulp); thread
+      // i < RH then writes row r0 + i's LSE.
+      const bool failed = !ok;
+      float inv[RH];
+      float lse_m = 0.f, lse_l = 0.f, lse_0 = -INFINITY;  // row r0 + i (i < RH)
 #pragma unroll
       for (int r = 0; r < RH; ++r) {
-        float v = l_part[r];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-        l_part[r] = v;
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < RH; ++r) lred[q4 * 32 + r0 + r] = l_part[r];
-      }
-      named_bar(2, ST);
-      // Row offsets come from shared memory: per-row index arithmetic here
-      // (a runtime division per row) made the store loop latency-bound.
-      const bool failed = !ok;
-      if (sid < NT) {
-        const float lt = lred[sid] + lred[32 + sid] + lred[64 + sid] + lred[96 + sid];
-        const bool live = lt > 0.f && !failed;
-        const long long row = rows[sid];
         // attention sink of the row's head (one split only; with splits the
         // merge adds it): one more exp2(sink) term in the denominator
-        const float sink =
-            a.num_splits == 1 && a.sinks && row >= 0 ? __ldg(a.sinks + row % a.Hq) : -INFINITY;
-        float inv = 0.f, res = failed ? -INFINITY : sink;
+        const float sink = a.num_splits == 1 ? sm_sink[r0 + r] : -INFINITY;
+        const float lt = lsum[r];
+        const bool live = lt > 0.f && !failed;
+        float mref = 0.f, l2 = 0.f;
+        inv[r] = 0.f;
         if (live) {
-          const float m = -sm_csm[sid].y;
-          float mref = m, l2 = lt, scl = 1.f;
+          const float m = -sm_csm[r0 + r].y;
+          float scl = 1.f;
+          mref = m;
+          l2 = lt;
           if (sink != -INFINITY) {
             const float sl = sink * kLog2e;
             mref = fmaxf(m, sl);
             scl = fast_exp2(m - mref);
             l2 = fmaf(lt, scl, fast_exp2(sl - mref));
           }
-          inv = a.v_scale * scl / l2;
-          res = (mref + log2f(l2)) * kLn2;
+          inv[r] = __fdividef(a.v_scale * scl, l2);
         }
-        sm_inv[sid] = inv;
+        if (i == r) {  // LSE = (mref + log2 l2) ln 2, else the sink alone, else -inf
+          lse_m = mref;
+          lse_l = l2;
+          lse_0 = failed ? -INFINITY : sink;
+        }
+      }
+      float* dst = a.num_splits == 1 ? a.out : a.o_part + (long long)split * rows_total * C::D;
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        const long long row = rows[r0 + r];
+        if (row >= 0) dst[row * C::D + i] = acc[r] * inv[r];
+      }
+      if (i < RH) {
+        const long long row = rows[r0 + i];
+        const float res = lse_l > 0.f ? (lse_m + log2f(lse_l)) * kLn2 : lse_0;
         if (row >= 0) {
           if (a.num_splits == 1) {
             if (a.lse) a.lse[row] = res;
@@ -1031,38 +1090,30 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           }
         }
       }
-      named_bar(2, ST);
-      float* dst = a.num_splits == 1 ? a.out : a.o_part + (long long)split * rows_total * C::D;
-#pragma unroll
-      for (int r = 0; r < RH; ++r) {
-        const long long row = rows[r0 + r];
-        if (row >= 0) dst[row * C::D + i] = acc[r] * sm_inv[r0 + r];
-      }
 
       // ---- fused merge (PDA_FLAG_FUSED_MERGE): the split that arrives last
-      // for these rows combines every split's partials by log-sum-exp --------
+      // for these rows combines every split's partials by log-sum-exp; each
+      // row group counts and merges its own rows --------------------------
       if (a.num_splits > 1 && a.fused_merge) {
         __threadfence();  // this split's partials are visible device-wide ...
-        named_bar(2, ST);
-        if (sid == 0) {   // ... before it counts itself in
-          int* ctr = a.merge_ctr + ((long long)d.b * a.Hkv + d.kvh) * a.row_tiles + d.rt;
-          *merge_flag = atomicAdd(ctr, 1) == a.num_splits - 1;
+        named_bar(gbar, GT);
+        if (i == 0) {     // ... before the group counts itself in
+          int* ctr = a.merge_ctr +
+                     (((long long)d.b * a.Hkv + d.kvh) * a.row_tiles + d.rt) * kMergeCtrPerGroup + grp;
+          merge_flag[grp] = atomicAdd(ctr, 1) == a.num_splits - 1;
         }
-        named_bar(2, ST);
-        if (*merge_flag) {
+        named_bar(gbar, GT);
+        if (merge_flag[grp]) {
           __threadfence();
           const int S = a.num_splits;  // <= 128
-          float* sm_lse = sm_inv;      // merged lse per row
-          // (1) per row: lse = m + ln sum_s exp(lse_s - m); warp w8 takes rows
-          // w8, w8 + 4 * SOFT_H, ...; lane l holds splits l, l + 32, l + 64, l + 96.
-          constexpr int NW8 = 4 * C::SOFT_H;
-          constexpr int RW = (NT + NW8 - 1) / NW8;
-          const int w8 = grp * 4 + q4;
+          // (1) per row: lse = m + ln sum_s exp(lse_s - m); warp q4 takes the
+          // group's rows q4, q4 + 4, ...; lane l holds splits l, l + 32, l + 64, l + 96.
+          constexpr int RW = (RH + 3) / 4;
           float v[RW][4];
 #pragma unroll
           for (int k = 0; k < RW; ++k) {
-            const int r = w8 + NW8 * k;
-            const long long row = r < NT ? rows[r] : -1;
+            const int rr = q4 + 4 * k;
+            const long long row = rr < RH ? rows[r0 + rr] : -1;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               const int spl = c * 32 + lane;
@@ -1073,9 +1124,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < RW; ++k) {
             // the row's attention sink is one more part: lse = sink, o = 0
-            const int rr = w8 + NW8 * k;
-            const long long rrow = rr < NT ? rows[rr] : -1;
-            const float sink = a.sinks && rrow >= 0 ? __ldg(a.sinks + rrow % a.Hq) : -INFINITY;
+            const int rr = q4 + 4 * k;
+            const long long rrow = rr < RH ? rows[r0 + rr] : -1;
+            const float sink = rrow >= 0 ? sm_sink[r0 + rr] : -INFINITY;
             float m = fmaxf(fmaxf(v[k][0], v[k][1]), fmaxf(v[k][2], v[k][3]));
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
@@ -1089,10 +1140,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
-            const int r = w8 + NW8 * k;
-            if (lane == 0 && r < NT) sm_lse[r] = m == -INFINITY ? -INFINITY : m + log2f(sum) * kLn2;
+            if (lane == 0 && rr < RH) sm_lse[r0 + rr] = m == -INFINITY ? -INFINITY : m + log2f(sum) * kLn2;
           }
-          named_bar(2, ST);
+          named_bar(gbar, GT);
           // (2) out[row, i] = sum_s exp(lse_s - lse) * o_s[row, i] over this
           // thread's rows; the rows' loads of one split go out together
 #pragma unroll
@@ -1116,11 +1166,11 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             const long long row = rows[r0 + r];
             if (row >= 0) a.out[row * C::D + i] = acc[r];
           }
-          if (sid < NT && rows[sid] >= 0 && a.lse) a.lse[rows[sid]] = sm_lse[sid];
+          if (i < RH && rows[r0 + i] >= 0 && a.lse) a.lse[rows[r0 + i]] = sm_lse[r0 + i];
         }
       }
-      named_bar(2, ST);  // item j's state and descriptor are no longer read
-      if (sid == 0) {
+      named_bar(gbar, GT);  // the group no longer reads item j's state and descriptor
+      if (i == 0) {
         mbar_arrive(&st_free[j & 1]);
         mbar_arrive(&desc_free[j & (C::DSLOTS - 1)]);
       }
