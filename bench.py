@@ -414,7 +414,9 @@ def run_ours(args, rank, world, local):
     achieved = alg_bytes / (avg_launch_ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     merge_launched = splits > 1 and not (kernel_name == "split_tma_kernel" and args.fused_merge)
-    launches_per_step = 1 + (1 if merge_launched else 0)
+    # the tensor-core kernel runs after its prologue kernel (counters, queue
+    # order, FP8 Q images); the merge kernel follows when splits are merged apart
+    launches_per_step = (2 if kernel_name == "split_tma_kernel" else 1) + (1 if merge_launched else 0)
 
     # Read-only HBM probe in the same run (our streaming-load kernel over a
     # 4 GiB buffer, larger than L2): the ceiling for a kernel that only reads.

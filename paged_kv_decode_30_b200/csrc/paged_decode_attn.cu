@@ -180,20 +180,33 @@ int choose_splits(const pda_params* p, const Plan& pl, int num_sms) {
 // partials follow (o_part then lse_part).
 struct WsLayout {
   size_t counters;  // bytes of the counter header (0 for the FMA kernel)
+  size_t order_off, qops_off;  // tensor-core kernel: queue order, FP8 Q images
   size_t o_off, lse_off, total;
 };
 constexpr size_t kMergeCtrOffset = 64;  // bytes: after the work-queue counters
+// Batches up to this size get a longest-first queue order (one CTA sorts
+// them); larger ones are handed out in sequence order.
+constexpr int kMaxOrderedBatch = 1 << 16;
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 
 WsLayout ws_layout(const pda_params* p, const Plan& pl, int splits) {
   WsLayout w{};
+  size_t end = 0;
   if (pl.tc) {
     const size_t groups = (size_t)p->batch * (size_t)p->num_kv_heads * (size_t)pl.row_tiles;
-    w.counters = round256(kMergeCtrOffset + groups * pda::kMergeCtrPerGroup * sizeof(int));
+    w.counters = kMergeCtrOffset + groups * pda::kMergeCtrPerGroup * sizeof(int);
+    w.order_off = round256(w.counters);
+    end = w.order_off + round256((size_t)p->batch * sizeof(int));
+    if (p->kv_dtype == PDA_KV_FP8_E4M3) {  // Q operand image + 32 row scales per group
+      const bool native = (p->flags & PDA_FLAG_NATIVE_FP8_QK) != 0;
+      const size_t qop = (size_t)(native ? pl.mt : 2 * pl.mt) * 128 + 128;
+      w.qops_off = end;
+      end += round256(groups * qop);
+    }
   }
-  w.o_off = w.lse_off = w.total = w.counters;
+  w.o_off = w.lse_off = w.total = end;
   if (splits > 1) {
     const size_t o_bytes = (size_t)splits * (size_t)pl.rows * (size_t)p->head_dim * sizeof(float);
     w.lse_off = w.o_off + round256(o_bytes);
@@ -355,12 +368,13 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
     }
     char* base = static_cast<char*>(ws);
     if (pl.tc) {
+      // the kernel's prologue zeroes the counters for this call, ranks the
+      // sequences into the queue order and writes the FP8 Q images
       a.sched = reinterpret_cast<int*>(base);
       a.merge_ctr = reinterpret_cast<int*>(base + kMergeCtrOffset);
-      // the counters start at zero for this call
-      const size_t used = kMergeCtrOffset + (size_t)p.batch * p.num_kv_heads * pl.row_tiles *
-                                                pda::kMergeCtrPerGroup * sizeof(int);
-      if (cudaMemsetAsync(base, 0, used, stream) != cudaSuccess) return PDA_ERR_CUDA;
+      a.header_words = (int)(wl.counters / sizeof(int));
+      a.order = p.batch <= kMaxOrderedBatch ? reinterpret_cast<int*>(base + wl.order_off) : nullptr;
+      a.qops = fp8 ? reinterpret_cast<uint8_t*>(base + wl.qops_off) : nullptr;
     }
     if (splits > 1) {
       a.o_part = reinterpret_cast<float*>(base + wl.o_off);
@@ -379,7 +393,7 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
     a.fused_merge = (p.flags & PDA_FLAG_FUSED_MERGE) != 0;
     const int grid = (int)std::min<long long>(items, dev->num_sms);
     e = launch_split_tma(kv, pl.mt, fp8 && (p.flags & PDA_FLAG_NATIVE_FP8_QK) != 0, k_pages,
-                         v_pages, a, grid, stream);
+                         v_pages, a, grid, stream, (p.flags & PDA_FLAG_NO_PDL) == 0);
   } else {
     const dim3 grid((unsigned)pl.row_tiles, (unsigned)(splits * p.num_kv_heads), (unsigned)p.batch);
     switch (p.head_dim) {

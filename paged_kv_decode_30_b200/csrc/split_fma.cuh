@@ -74,11 +74,14 @@ struct SplitArgs {
   float v_scale;             // 1, or kv_scale for FP8
   long long page_stride;     // bytes per page: Hkv * P * D * elt
   long long head_stride;     // bytes per (page, head) block: P * D * elt
-  // persistent tensor-core kernel only (counters zeroed by the host just
-  // before the launch, in stream order):
+  // persistent tensor-core kernel only (prepared by its prologue kernel,
+  // which runs just before it on the same stream):
   int* sched;                // [0] next work item
   int* merge_ctr;            // [B * Hkv * row_tiles * kMergeCtrPerGroup] splits finished
                              // per (group, softmax row group)
+  int header_words;          // ints from sched to the end of merge_ctr (zeroed first)
+  int* order;                // [B] sequences, most visible tiles first: the queue order
+  uint8_t* qops;             // FP8: Q operand image + row scales per (b, kvh, row tile)
   int num_items;             // B * Hkv * num_splits * row_tiles
   const float* sinks;        // [Hq] attention-sink logit per query head, or null
   int fused_merge;           // 1: the last split of a group merges it in-kernel

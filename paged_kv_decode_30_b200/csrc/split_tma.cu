@@ -2,6 +2,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <mutex>
 
 #include "split_tma.cuh"
@@ -47,7 +48,7 @@ bool make_pool_map(CUtensorMap* map, const void* base, long long rows, int elt, 
 
 template <int KV, int NT, bool QN = false>
 cudaError_t launch_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const SplitArgs& a,
-                       int grid, cudaStream_t stream) {
+                       int grid, cudaStream_t stream, bool pdl) {
   using C = TmaCfg<KV, NT, QN>;
   auto kern = split_tma_kernel<KV, NT, QN>;
   static unsigned long long attr_set = 0;  // bit d: opt-in set on device d (< 64)
@@ -60,15 +61,30 @@ cudaError_t launch_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const Split
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
   }
-  kern<<<dim3((unsigned)grid), C::THREADS, C::SMEM_ALLOC, stream>>>(mk, mv, a);
-  return cudaGetLastError();
+  // prologue: block 0 (counters, queue order), FP8 one block per Q image
+  const long long q_blocks = KV ? (long long)a.B * a.Hkv * a.row_tiles : 0;
+  if (q_blocks >= INT_MAX) return cudaErrorInvalidValue;
+  split_tma_prologue<KV, NT, QN><<<dim3((unsigned)(1 + q_blocks)), 256, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, mk, mv, a);
 }
 
 }  // namespace
 
 cudaError_t launch_split_tma(int kv, int nt, bool native_qk, const void* k_pages,
                              const void* v_pages, const SplitArgs& a, int grid,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, bool pdl) {
   const long long rows = (long long)a.num_pages * a.Hkv * a.page_size;
   const int elt = kv == 0 ? 2 : 1;
   const int box_rows = a.page_size < 128 ? a.page_size : 128;
@@ -78,21 +94,21 @@ cudaError_t launch_split_tma(int kv, int nt, bool native_qk, const void* k_pages
     return cudaErrorInvalidValue;
   if (kv == 0) {
     switch (nt) {
-      case 4: return launch_cfg<0, 4>(mk, mv, a, grid, stream);
-      case 8: return launch_cfg<0, 8>(mk, mv, a, grid, stream);
+      case 4: return launch_cfg<0, 4>(mk, mv, a, grid, stream, pdl);
+      case 8: return launch_cfg<0, 8>(mk, mv, a, grid, stream, pdl);
       default: return cudaErrorNotSupported;
     }
   }
   if (native_qk) {
     switch (nt) {
-      case 16: return launch_cfg<1, 16, true>(mk, mv, a, grid, stream);
-      case 32: return launch_cfg<1, 32, true>(mk, mv, a, grid, stream);
+      case 16: return launch_cfg<1, 16, true>(mk, mv, a, grid, stream, pdl);
+      case 32: return launch_cfg<1, 32, true>(mk, mv, a, grid, stream, pdl);
       default: return cudaErrorNotSupported;
     }
   }
   switch (nt) {
-    case 16: return launch_cfg<1, 16>(mk, mv, a, grid, stream);
-    case 32: return launch_cfg<1, 32>(mk, mv, a, grid, stream);
+    case 16: return launch_cfg<1, 16>(mk, mv, a, grid, stream, pdl);
+    case 32: return launch_cfg<1, 32>(mk, mv, a, grid, stream, pdl);
     default: return cudaErrorNotSupported;
   }
 }

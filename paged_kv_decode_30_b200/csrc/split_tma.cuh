@@ -87,6 +87,9 @@ struct TmaCfg {
   static constexpr int Q_BYTES = Q_ROWS * D * (BF16 ? 2 : 1);
   static constexpr int Q_HALF = (Q_ROWS / 8) * 1024;  // bf16: 64-element half of each row
   static constexpr int Q_BUF = ((Q_BYTES + 1023) / 1024) * 1024;  // one of two Q buffers
+  // FP8: the prologue kernel's Q operand image of one (b, kv head, row tile)
+  // in global memory: Q_BYTES as the MMA reads them, then 32 row scales
+  static constexpr int QOP = Q_BYTES + 128;
   static constexpr int P_ROW = N2 * ELT;               // bytes per token row of P^T
   static constexpr int P_SBO = 8 * P_ROW;
   static constexpr int P_BYTES = (TILE / 8) * P_SBO;
@@ -231,6 +234,8 @@ __device__ __forceinline__ bool mbar_ready(uint64_t* bar, uint32_t parity) {
 
 // Item t of the queue -> (b, kvh, split, rt); rt varies fastest, so the
 // splits of one group are drawn close together and their merge comes early.
+// Sequences come in the prologue's order (most visible tiles first), so the
+// queue ends on short items and the CTAs finish close together.
 __device__ __forceinline__ void decode_item(const SplitArgs& a, int t, int& b, int& kvh,
                                             int& split, int& rt) {
   rt = t % a.row_tiles;
@@ -239,6 +244,7 @@ __device__ __forceinline__ void decode_item(const SplitArgs& a, int t, int& b, i
   u /= a.num_splits;
   kvh = u % a.Hkv;
   b = u / a.Hkv;
+  if (a.order) b = __ldcg(a.order + b);
 }
 
 template <int KV, int NT, bool QN = false>
@@ -324,6 +330,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
   __syncthreads();
   tmem_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above overlaps the prologue kernel; the counters, the queue
+  // order and the Q images it writes are read only after this.
+  pdl_wait_primary();
 
   if (warp == C::SCHED) {
     // ======================= scheduler (whole warp) ==========================
@@ -400,12 +409,13 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       mbar_arrive(&desc_full[j & (C::DSLOTS - 1)]);
       return more;
     };
-    // Q rows of an item are prefetched into L2 when the item is published
-    // (one bulk prefetch per query row position: its G heads are contiguous),
-    // so preparing its Q operand later reads L2, not HBM.
+    // bf16: Q rows of an item are prefetched into L2 when the item is
+    // published (one bulk prefetch per query row position: its G heads are
+    // contiguous), so preparing its Q operand later reads L2, not HBM. (FP8
+    // copies the prologue kernel's image instead.)
     auto prefetch_q = [&](int j) {
       const Desc& d = descs[j & (C::DSLOTS - 1)];
-      if (lane < a.Lq) {
+      if (C::BF16 && lane < a.Lq) {
         const uint16_t* src = a.q + ((long long)(d.b * a.Lq + lane) * a.Hq + d.kvh * a.G) * C::D;
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src),
                      "r"((uint32_t)(a.G * C::D * 2))
@@ -461,63 +471,15 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
                                       (n & 7) * 128 + (((jj & 7) ^ (n & 7)) << 4)) = qv[k];
         }
         if (lane < NT) cs[lane] = a.qk_scale_log2;
-      } else if (lane < NT) {
-        // Lane n: the hi and lo operand rows of item row n in e4m3, 128 bytes each,
-        // SW128 K-major. q * 2^e2 = hi + lo / 16 exactly, with 2^e2 the power
-        // of two that puts max|q| of the row in [128, 256). Native QK keeps
-        // hi alone (q quantised to e4m3 at that scale).
-        const int n = lane, R = R0 + n;
-        const bool live = R < a.M;
-        const uint4* src = reinterpret_cast<const uint4*>(a.q);
-        if (live) {
-          const int qi = R / a.G, h = kvh * a.G + R % a.G;
-          src = reinterpret_cast<const uint4*>(a.q + ((long long)(b * a.Lq + qi) * a.Hq + h) * C::D);
+      } else {
+        // the prologue kernel's image of this (b, kv head, row tile): one bulk
+        // copy, counted on q_ready next to the 32 lanes' arrivals below
+        const uint8_t* img = a.qops + (((long long)b * a.Hkv + kvh) * a.row_tiles + d.rt) * C::QOP;
+        if (lane == 0) {
+          mbar_expect_tx(&q_ready[j & 1], C::Q_BYTES);
+          bulk_g2s(qbuf, img, C::Q_BYTES, &q_ready[j & 1]);
         }
-        float mx = 0.f;
-        if (live) {  // pass 1: max |q| of the row, 8 loads in flight
-#pragma unroll 8
-          for (int k = 0; k < 16; ++k) {
-            float g8[8];
-            bf16x8_to_f32(__ldg(src + k), g8);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(g8[e]));
-          }
-        }
-        const int e2 = mx > 0.f ? 8 - ilogbf(mx) - 1 : 0;  // mx * 2^e2 < 256 <= 448
-        const float sc = ldexpf(1.f, e2);
-        cs[n] = ldexpf(a.qk_scale_log2, -e2);
-        // operand rows in row-group order: hi of row n at 16 (n / 8) + n % 8,
-        // its lo 8 rows later (native QK: hi of row n at n)
-        const int rh = C::QN_ ? n : 16 * (n >> 3) + (n & 7), rl = rh + 8;
-#pragma unroll 2
-        for (int c = 0; c < 8; ++c) {  // pass 2 (L1 hits): 16 elements -> a chunk of hi and of lo
-          float f[16];
-          const uint4 u0 = live ? __ldg(src + 2 * c) : make_uint4(0, 0, 0, 0);
-          const uint4 u1 = live ? __ldg(src + 2 * c + 1) : make_uint4(0, 0, 0, 0);
-          bf16x8_to_f32(u0, *reinterpret_cast<float(*)[8]>(f));
-          bf16x8_to_f32(u1, *reinterpret_cast<float(*)[8]>(f + 8));
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t hv = 0, lv = 0;
-#pragma unroll
-            for (int e = 0; e < 4; e += 2) {
-              const float x0 = f[4 * w + e] * sc, x1 = f[4 * w + e + 1] * sc;
-              const uint32_t h2 = f32x2_to_e4m3x2(x0, x1);
-              const float r0 = (x0 - e4m3_to_f32(h2)) * 16.f;
-              const float r1 = (x1 - e4m3_to_f32(h2 >> 8)) * 16.f;
-              hv |= h2 << (8 * e);
-              lv |= f32x2_to_e4m3x2(r0, r1) << (8 * e);
-            }
-            hw[w] = hv;
-            lw[w] = lv;
-          }
-          *reinterpret_cast<uint4*>(qbuf + (rh >> 3) * 1024 + (rh & 7) * 128 +
-                                    ((c ^ (rh & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          if constexpr (!C::QN_)
-            *reinterpret_cast<uint4*>(qbuf + (rl >> 3) * 1024 + (rl & 7) * 128 +
-                                      ((c ^ (rl & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
+        if (lane < NT) cs[lane] = __ldcg(reinterpret_cast<const float*>(img + C::Q_BYTES) + lane);
       }
       fence_proxy_async_smem();  // the Q operand is read by the tensor core
       __syncwarp();
@@ -1189,11 +1151,133 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
   }
 }
 
-// Host launcher (split_tma.cu). kv: 0 bf16, 1 e4m3; nt: rows per CTA;
-// native_qk: FP8 with one-term e4m3 Q; grid: persistent CTAs (at most one
-// per SM).
+// Buckets of the prologue's counting sort: sequences with this many or more
+// visible tiles share the last one.
+constexpr int kOrderBuckets = 1024;
+
+// Prologue of split_tma_kernel, launched just before it on the same stream
+// (the main kernel waits for it with griddepcontrol.wait):
+//  * block 0 zeroes the counter header, then ranks the sequences by their
+//    visible 128-token tiles, most first (a counting sort; ties in any
+//    order: an item's result does not depend on the CTA that runs it), into
+//    a.order, the order in which the work queue hands them out;
+//  * FP8, blocks 1.. : the Q operand of one (b, kv head, row tile) each,
+//    written as the S^T MMA reads it (the same scale choice and two-term
+//    split as the in-kernel path), then its 32 row scales.
+template <int KV, int NT, bool QN = false>
+__global__ void __launch_bounds__(256) split_tma_prologue(const SplitArgs a) {
+  using C = TmaCfg<KV, NT, QN>;
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  pdl_launch_dependents();  // the main kernel may start its own set-up now
+  const int tid = threadIdx.x;
+  if (blockIdx.x == 0) {
+    __shared__ int hist[kOrderBuckets];
+    __shared__ int wsum[8];
+    for (int w = tid; w < a.header_words; w += 256) a.sched[w] = 0;
+    if (a.order == nullptr) return;
+    for (int k = tid; k < kOrderBuckets; k += 256) hist[k] = 0;
+    __syncthreads();
+    const int Lmax = a.max_pages << a.log2_page;
+    auto bucket = [&](int b) {  // descending visible tiles -> ascending bucket
+      const int L = min(max(__ldg(a.kv_lens + b), 0), Lmax);
+      int lo, hi0, lo1, hi;
+      row_range(a, L, 0, lo, hi0);        // first query row: the union's start
+      row_range(a, L, a.Lq - 1, lo1, hi);  // last query row: the union's end
+      const int n = hi > lo ? (hi + C::TILE - 1) / C::TILE - lo / C::TILE : 0;
+      return kOrderBuckets - 1 - min(n, kOrderBuckets - 1);
+    };
+    for (int b = tid; b < a.B; b += 256) atomicAdd(&hist[bucket(b)], 1);
+    __syncthreads();
+    // exclusive scan of the histogram: 4 buckets per thread, then warps
+    constexpr int PT = kOrderBuckets / 256;
+    int v[PT], own = 0;
+#pragma unroll
+    for (int k = 0; k < PT; ++k) {
+      v[k] = hist[tid * PT + k];
+      own += v[k];
+    }
+    const int lane = tid & 31, warp = tid >> 5;
+    int inc = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(FULL, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += wsum[w];
+    int run = base + inc - own;
+#pragma unroll
+    for (int k = 0; k < PT; ++k) {
+      hist[tid * PT + k] = run;
+      run += v[k];
+    }
+    __syncthreads();
+    for (int b = tid; b < a.B; b += 256) a.order[atomicAdd(&hist[bucket(b)], 1)] = b;
+    return;
+  }
+  if constexpr (!C::BF16) {
+    // item q = (b, kvh, rt), rt fastest; thread: row n = tid / 8, 16-element
+    // chunk c = tid % 8 of it (the 8 threads of a row are adjacent lanes)
+    const int q = blockIdx.x - 1;
+    const int rt = q % a.row_tiles, kvh = (q / a.row_tiles) % a.Hkv, b = q / (a.row_tiles * a.Hkv);
+    uint8_t* img = a.qops + (long long)q * C::QOP;
+    const int n = tid >> 3, c = tid & 7;
+    if (n >= NT) return;  // whole groups of 8 lanes
+    const int R = rt * NT + n;
+    const bool live = R < a.M;
+    float f[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) f[e] = 0.f;
+    if (live) {
+      const int qi = R / a.G, h = kvh * a.G + R % a.G;
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((long long)(b * a.Lq + qi) * a.Hq + h) * C::D);
+      bf16x8_to_f32(__ldg(src + 2 * c), *reinterpret_cast<float(*)[8]>(f));
+      bf16x8_to_f32(__ldg(src + 2 * c + 1), *reinterpret_cast<float(*)[8]>(f + 8));
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(f[e]));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+    // q * 2^e2 = hi + lo / 16 exactly, with 2^e2 the power of two that puts
+    // max|q| of the row in [128, 256) (native QK: hi alone)
+    const int e2 = mx > 0.f ? 8 - ilogbf(mx) - 1 : 0;
+    const float sc = ldexpf(1.f, e2);
+    if (c == 0) reinterpret_cast<float*>(img + C::Q_BYTES)[n] = ldexpf(a.qk_scale_log2, -e2);
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t hv = 0, lv = 0;
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const float x0 = f[4 * w + e] * sc, x1 = f[4 * w + e + 1] * sc;
+        const uint32_t h2 = f32x2_to_e4m3x2(x0, x1);
+        const float r0 = (x0 - e4m3_to_f32(h2)) * 16.f;
+        const float r1 = (x1 - e4m3_to_f32(h2 >> 8)) * 16.f;
+        hv |= h2 << (8 * e);
+        lv |= f32x2_to_e4m3x2(r0, r1) << (8 * e);
+      }
+      hw[w] = hv;
+      lw[w] = lv;
+    }
+    // operand rows in row-group order (as the in-kernel path writes them)
+    const int rh = C::QN_ ? n : 16 * (n >> 3) + (n & 7), rl = rh + 8;
+    *reinterpret_cast<uint4*>(img + (rh >> 3) * 1024 + (rh & 7) * 128 + ((c ^ (rh & 7)) << 4)) =
+        make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    if constexpr (!C::QN_)
+      *reinterpret_cast<uint4*>(img + (rl >> 3) * 1024 + (rl & 7) * 128 + ((c ^ (rl & 7)) << 4)) =
+          make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+// Host launcher (split_tma.cu): the prologue kernel, then split_tma_kernel
+// (its programmatic dependent when pdl). kv: 0 bf16, 1 e4m3; nt: rows per
+// CTA; native_qk: FP8 with one-term e4m3 Q; grid: persistent CTAs (at most
+// one per SM).
 cudaError_t launch_split_tma(int kv, int nt, bool native_qk, const void* k_pages,
                              const void* v_pages, const SplitArgs& a, int grid,
-                             cudaStream_t stream);
+                             cudaStream_t stream, bool pdl);
 
 }  // namespace pda

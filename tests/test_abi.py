@@ -160,8 +160,8 @@ def test_workspace_bytes(lib):
     assert B.workspace_bytes(headline_params(num_splits=1, flags=B.PDA_FLAG_CUDA_CORES)) == 0
     # tensor-core kernel: a counter header (the work-queue counter, then four
     # split-arrival counters per (sequence, kv head, row tile): one per softmax
-    # row group) before the partials
-    header = (64 + 128 * 8 * 4 * 4 + 255) // 256 * 256
+    # row group) and the queue order (one int per sequence) before the partials
+    header = (64 + 128 * 8 * 4 * 4 + 255) // 256 * 256 + (128 * 4 + 255) // 256 * 256
     assert B.workspace_bytes(headline_params(num_splits=1)) == header
     got = B.workspace_bytes(headline_params(num_splits=4))
     assert got >= header + expect_o + 4 * rows * 4 and got < header + expect_o + 4 * rows * 4 + 512
