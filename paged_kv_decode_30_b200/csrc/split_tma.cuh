@@ -738,7 +738,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     float* wmax = reinterpret_cast<float*>(smem + C::OFF_WMAX);
     float* sm_alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
     float* lred = reinterpret_cast<float*>(smem + C::OFF_LRED);
-    float* sm_lse = reinterpret_cast<float*>(smem + C::OFF_INV);
+    float* sm_lse = reinterpret_cast<float*>(smem + C::OFF_INV);  // fused merge (reuses sm_inv)
     const long long rows_total = (long long)a.B * a.Lq * a.Hq;
     constexpr float kLn2 = 0.69314718055994531f, kLog2e = 1.4426950408889634f;
     // this thread's column offset in an S^T / O^T / row-sum region
@@ -880,16 +880,22 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           // barrier then stops all four of its warps together.
           if (n > 0) {
             if (wait_o(g - 1)) {
-              float o[16];
-              tmem_ld16_raw(o_tm, o);
+              if constexpr (C::BF16) {
+                float o[16];
+                tmem_ld16_raw(o_tm, o);
 #pragma unroll
-              for (int c = 0; c < 16; ++c) o[c] *= al[C::BF16 ? (c % NT) : (c % RH)];
-              tmem_st16(o_tm, o);
-              if constexpr (!C::BF16) {
-                tmem_ld16_raw(l_tm, o);
+                for (int c = 0; c < 16; ++c) o[c] *= al[c % NT];
+                tmem_st16(o_tm, o);
+              } else {  // 8 columns at a time (O hi, O lo, sums hi, sums lo)
+#pragma unroll 1
+                for (int part = 0; part < 4; ++part) {
+                  const uint32_t ta = (part < 2 ? o_tm : l_tm) + (part & 1) * RH;
+                  float o[RH];
+                  tmem_ld8(ta, o);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) o[c] *= al[c % RH];
-                tmem_st16(l_tm, o);
+                  for (int c = 0; c < RH; ++c) o[c] *= al[c];
+                  tmem_st8(ta, o);
+                }
               }
               tmem_fence_before();
             } else {
@@ -1001,49 +1007,35 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         for (int r = 0; r < RH; ++r)
           lsum[r] = lred[r0 + r] + lred[32 + r0 + r] + lred[64 + r0 + r] + lred[96 + r0 + r];
       }
-      // Every thread derives its rows' normalisers itself (the inputs are the
-      // same for all of them; an approximate division, 2 ulp); thread
-      // i < RH then writes row r0 + i's LSE.
+      // Thread i < RH derives row r0 + i's normaliser and LSE (the row sum
+      // is in every thread: FP8 from TMEM, bf16 from the reduction above)
+      // and shares the normaliser through shared memory.
       const bool failed = !ok;
-      float inv[RH];
-      float lse_m = 0.f, lse_l = 0.f, lse_0 = -INFINITY;  // row r0 + i (i < RH)
+      float* sm_inv = reinterpret_cast<float*>(smem + C::OFF_INV);
+      if (i < RH) {
+        float lt = 0.f;
 #pragma unroll
-      for (int r = 0; r < RH; ++r) {
+        for (int r = 0; r < RH; ++r)
+          if (r == i) lt = lsum[r];
+        const int rr = r0 + i;
+        const long long row = rows[rr];
         // attention sink of the row's head (one split only; with splits the
         // merge adds it): one more exp2(sink) term in the denominator
-        const float sink = a.num_splits == 1 ? sm_sink[r0 + r] : -INFINITY;
-        const float lt = lsum[r];
-        const bool live = lt > 0.f && !failed;
-        float mref = 0.f, l2 = 0.f;
-        inv[r] = 0.f;
-        if (live) {
-          const float m = -sm_csm[r0 + r].y;
-          float scl = 1.f;
-          mref = m;
-          l2 = lt;
+        const float sink = a.num_splits == 1 ? sm_sink[rr] : -INFINITY;
+        float inv = 0.f, res = failed ? -INFINITY : sink;
+        if (lt > 0.f && !failed) {
+          const float m = -sm_csm[rr].y;
+          float mref = m, l2 = lt, scl = 1.f;
           if (sink != -INFINITY) {
             const float sl = sink * kLog2e;
             mref = fmaxf(m, sl);
             scl = fast_exp2(m - mref);
             l2 = fmaf(lt, scl, fast_exp2(sl - mref));
           }
-          inv[r] = __fdividef(a.v_scale * scl, l2);
+          inv = a.v_scale * scl / l2;
+          res = (mref + log2f(l2)) * kLn2;
         }
-        if (i == r) {  // LSE = (mref + log2 l2) ln 2, else the sink alone, else -inf
-          lse_m = mref;
-          lse_l = l2;
-          lse_0 = failed ? -INFINITY : sink;
-        }
-      }
-      float* dst = a.num_splits == 1 ? a.out : a.o_part + (long long)split * rows_total * C::D;
-#pragma unroll
-      for (int r = 0; r < RH; ++r) {
-        const long long row = rows[r0 + r];
-        if (row >= 0) dst[row * C::D + i] = acc[r] * inv[r];
-      }
-      if (i < RH) {
-        const long long row = rows[r0 + i];
-        const float res = lse_l > 0.f ? (lse_m + log2f(lse_l)) * kLn2 : lse_0;
+        sm_inv[rr] = inv;
         if (row >= 0) {
           if (a.num_splits == 1) {
             if (a.lse) a.lse[row] = res;
@@ -1052,13 +1044,20 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           }
         }
       }
+      named_bar(gbar, GT);
+      float* dst = a.num_splits == 1 ? a.out : a.o_part + (long long)split * rows_total * C::D;
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        const long long row = rows[r0 + r];
+        if (row >= 0) dst[row * C::D + i] = acc[r] * sm_inv[r0 + r];
+      }
 
       // ---- fused merge (PDA_FLAG_FUSED_MERGE): the split that arrives last
       // for these rows combines every split's partials by log-sum-exp; each
       // row group counts and merges its own rows --------------------------
       if (a.num_splits > 1 && a.fused_merge) {
         __threadfence();  // this split's partials are visible device-wide ...
-        named_bar(gbar, GT);
+        named_bar(gbar, GT);  // (and every sm_inv read is done: sm_lse reuses it)
         if (i == 0) {     // ... before the group counts itself in
           int* ctr = a.merge_ctr +
                      (((long long)d.b * a.Hkv + d.kvh) * a.row_tiles + d.rt) * kMergeCtrPerGroup + grp;
