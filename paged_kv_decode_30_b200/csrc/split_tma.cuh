@@ -744,43 +744,241 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     // this thread's column offset in an S^T / O^T / row-sum region
     const uint32_t col_s = C::BF16 ? 0 : (C::QN_ ? r0 : 2 * r0);
     const uint32_t col_o = C::BF16 ? 0 : 2 * r0;
-    int g = 0;  // tiles of this CTA so far (over all items)
-    bool ok = true;
-    for (int j = 0; ok; ++j) {
-      ok = !*abort_flag && mbar_wait(&desc_full[j & (C::DSLOTS - 1)], (j / C::DSLOTS) & 1, a.err);
-      if (ok && descs[j & (C::DSLOTS - 1)].b >= 0) ok = mbar_wait(&q_ready[j & 1], (j >> 1) & 1, a.err);
-      if (!named_bar_and(gbar, GT, ok)) {
-        ok = false;
-        break;
+    // wait until the O^T MMAs of tile k have completed (all lanes agree)
+    auto wait_o = [&](int k) -> bool {
+      const bool ok_w = __all_sync(FULL, mbar_wait(&o_full[k & 1], (k >> 1) & 1, a.err));
+      if (ok_w) tmem_fence_after();
+      return ok_w;
+    };
+    // Epilogue of item jj (last tile g_last, nt tiles, status ok_in; lp: bf16
+    // partial row sums): reads O^T (FP8: and the row sums) from TMEM region
+    // jj & 1 and releases it, normalises, stores O and the LSE (or the
+    // split's partials), runs the fused merge and releases the item's state
+    // slot and descriptor. It runs after the next item's first tile, when
+    // item jj's last MMAs are long done. Returns the group's agreement that
+    // nothing failed.
+    auto epilogue = [&](int jj, int g_last, int nt, bool ok_in, const float* lp) -> bool {
+      const Desc& dd = descs[jj & (C::DSLOTS - 1)];
+      const int split = dd.split;
+      const uint8_t* sl = slot_of(jj);
+      const long long* rows = reinterpret_cast<const long long*>(sl + C::SL_ROWS);
+      const float2* sm_csm = reinterpret_cast<const float2*>(sl + C::SL_CSM);
+      const float* sm_sink = reinterpret_cast<const float*>(sl + C::SL_SINK);
+      const uint32_t o_tm = tmem + lane_off + C::COL_O + (jj & 1) * C::N2 + col_o;
+      const uint32_t l_tm = tmem + lane_off + C::COL_L + (jj & 1) * C::N2 + col_o;
+      float acc[RH], lsum[RH];
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        acc[r] = 0.f;
+        lsum[r] = 0.f;
       }
+      bool e_ok = ok_in;
+      if (__all_sync(FULL, e_ok && nt > 0 && !*abort_flag)) {
+        e_ok = wait_o(g_last);
+        if (e_ok) {
+          float o[16];
+          tmem_ld16_raw(o_tm, o);
+          if constexpr (C::BF16) {
+#pragma unroll
+            for (int r = 0; r < RH; ++r) acc[r] = o[r] + o[NT + r];  // P = P_hi + P_lo
+          } else {
+#pragma unroll
+            for (int r = 0; r < RH; ++r) acc[r] = fmaf(o[RH + r], 0.0625f, o[r]);  // P_hi + (16 P_lo) / 16
+            tmem_ld16_raw(l_tm, o);
+#pragma unroll
+            for (int r = 0; r < RH; ++r) lsum[r] = fmaf(o[RH + r], 0.0625f, o[r]);
+          }
+        }
+      }
+      tmem_fence_before();
+      mbar_arrive(&o_free[jj & 1]);  // region jj & 1 may take item jj + 2
+      const bool eok = named_bar_and(gbar, GT, e_ok);
+      if (!eok) *abort_flag = 1;
+
+      // ---- epilogue: normaliser and LSE per row, then the O rows ----------
+      if constexpr (C::BF16) {
+        // row sums: over the lanes, then over the group's four warps
+#pragma unroll
+        for (int r = 0; r < RH; ++r) {
+          float v = lp[r];
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+          lsum[r] = v;
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int r = 0; r < RH; ++r) lred[q4 * 32 + r0 + r] = lsum[r];
+        }
+        named_bar(gbar, GT);
+#pragma unroll
+        for (int r = 0; r < RH; ++r)
+          lsum[r] = lred[r0 + r] + lred[32 + r0 + r] + lred[64 + r0 + r] + lred[96 + r0 + r];
+      }
+      // Thread i < RH derives row r0 + i's normaliser and LSE (the row sum
+      // is in every thread: FP8 from TMEM, bf16 from the reduction above)
+      // and shares the normaliser through shared memory.
+      const bool failed = !eok;
+      float* sm_inv = reinterpret_cast<float*>(smem + C::OFF_INV);
+      if (i < RH) {
+        float lt = 0.f;
+#pragma unroll
+        for (int r = 0; r < RH; ++r)
+          if (r == i) lt = lsum[r];
+        const int rr = r0 + i;
+        const long long row = rows[rr];
+        // attention sink of the row's head (one split only; with splits the
+        // merge adds it): one more exp2(sink) term in the denominator
+        const float sink = a.num_splits == 1 ? sm_sink[rr] : -INFINITY;
+        float inv = 0.f, res = failed ? -INFINITY : sink;
+        if (lt > 0.f && !failed) {
+          const float m = -sm_csm[rr].y;
+          float mref = m, l2 = lt, scl = 1.f;
+          if (sink != -INFINITY) {
+            const float sink2 = sink * kLog2e;
+            mref = fmaxf(m, sink2);
+            scl = fast_exp2(m - mref);
+            l2 = fmaf(lt, scl, fast_exp2(sink2 - mref));
+          }
+          inv = a.v_scale * scl / l2;
+          res = (mref + log2f(l2)) * kLn2;
+        }
+        sm_inv[rr] = inv;
+        if (row >= 0) {
+          if (a.num_splits == 1) {
+            if (a.lse) a.lse[row] = res;
+          } else {
+            a.lse_part[(long long)split * rows_total + row] = res;
+          }
+        }
+      }
+      named_bar(gbar, GT);
+      float* dst = a.num_splits == 1 ? a.out : a.o_part + (long long)split * rows_total * C::D;
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        const long long row = rows[r0 + r];
+        if (row >= 0) dst[row * C::D + i] = acc[r] * sm_inv[r0 + r];
+      }
+
+      // ---- fused merge (PDA_FLAG_FUSED_MERGE): the split that arrives last
+      // for these rows combines every split's partials by log-sum-exp; each
+      // row group counts and merges its own rows --------------------------
+      if (a.num_splits > 1 && a.fused_merge) {
+        __threadfence();  // this split's partials are visible device-wide ...
+        named_bar(gbar, GT);  // (and every sm_inv read is done: sm_lse reuses it)
+        if (i == 0) {     // ... before the group counts itself in
+          int* ctr = a.merge_ctr +
+                     (((long long)dd.b * a.Hkv + dd.kvh) * a.row_tiles + dd.rt) * kMergeCtrPerGroup + grp;
+          merge_flag[grp] = atomicAdd(ctr, 1) == a.num_splits - 1;
+        }
+        named_bar(gbar, GT);
+        if (merge_flag[grp]) {
+          __threadfence();
+          const int S = a.num_splits;  // <= 128
+          // (1) per row: lse = m + ln sum_s exp(lse_s - m); warp q4 takes the
+          // group's rows q4, q4 + 4, ...; lane l holds splits l, l + 32, l + 64, l + 96.
+          constexpr int RW = (RH + 3) / 4;
+          float v[RW][4];
+#pragma unroll
+          for (int k = 0; k < RW; ++k) {
+            const int rr = q4 + 4 * k;
+            const long long row = rr < RH ? rows[r0 + rr] : -1;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int spl = c * 32 + lane;
+              v[k][c] = row >= 0 && spl < S ? __ldcg(a.lse_part + (long long)spl * rows_total + row)
+                                            : -INFINITY;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < RW; ++k) {
+            // the row's attention sink is one more part: lse = sink, o = 0
+            const int rr = q4 + 4 * k;
+            const long long rrow = rr < RH ? rows[r0 + rr] : -1;
+            const float sink = rrow >= 0 ? sm_sink[r0 + rr] : -INFINITY;
+            float m = fmaxf(fmaxf(v[k][0], v[k][1]), fmaxf(v[k][2], v[k][3]));
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+            m = fmaxf(m, sink);
+            float sum = 0.f;
+            if (m != -INFINITY) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                if (v[k][c] != -INFINITY) sum += fast_exp2((v[k][c] - m) * kLog2e);
+              if (lane == 0 && sink != -INFINITY) sum += fast_exp2((sink - m) * kLog2e);
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
+            if (lane == 0 && rr < RH) sm_lse[r0 + rr] = m == -INFINITY ? -INFINITY : m + log2f(sum) * kLn2;
+          }
+          named_bar(gbar, GT);
+          // (2) out[row, i] = sum_s exp(lse_s - lse) * o_s[row, i] over this
+          // thread's rows; the rows' loads of one split go out together
+#pragma unroll
+          for (int r = 0; r < RH; ++r) acc[r] = 0.f;
+          for (int spl = 0; spl < S; ++spl) {
+            float ls[RH], ov[RH];
+#pragma unroll
+            for (int r = 0; r < RH; ++r) {
+              const long long row = rows[r0 + r];
+              const long long idx = (long long)spl * rows_total + (row >= 0 ? row : 0);
+              ls[r] = row >= 0 ? __ldcg(a.lse_part + idx) : -INFINITY;
+              ov[r] = row >= 0 ? __ldcg(a.o_part + idx * C::D + i) : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < RH; ++r)
+              if (ls[r] != -INFINITY)
+                acc[r] = fmaf(fast_exp2((ls[r] - sm_lse[r0 + r]) * kLog2e), ov[r], acc[r]);
+          }
+#pragma unroll
+          for (int r = 0; r < RH; ++r) {
+            const long long row = rows[r0 + r];
+            if (row >= 0) a.out[row * C::D + i] = acc[r];
+          }
+          if (i < RH && rows[r0 + i] >= 0 && a.lse) a.lse[rows[r0 + i]] = sm_lse[r0 + i];
+        }
+      }
+      named_bar(gbar, GT);  // the group no longer reads item jj's state and descriptor
+      if (i == 0) {
+        mbar_arrive(&st_free[jj & 1]);
+        mbar_arrive(&desc_free[jj & (C::DSLOTS - 1)]);
+      }
+      return eok;
+    };
+
+    int g = 0;  // tiles of this CTA so far (over all items)
+    bool ok = true, acc_prev = true;
+    // the item whose epilogue is pending (-1: none), its last tile, tile
+    // count, status and (bf16) partial row sums
+    int pend = -1, pend_g = 0, pend_nt = 0;
+    bool pend_ok = true;
+    float l_pend[RH];
+#pragma unroll
+    for (int r = 0; r < RH; ++r) l_pend[r] = 0.f;
+    for (int j = 0;; ++j) {
+      bool w = acc_prev && !*abort_flag &&
+               mbar_wait(&desc_full[j & (C::DSLOTS - 1)], (j / C::DSLOTS) & 1, a.err);
+      if (w && descs[j & (C::DSLOTS - 1)].b >= 0) w = mbar_wait(&q_ready[j & 1], (j >> 1) & 1, a.err);
+      if (!named_bar_and(gbar, GT, w)) ok = false;
       const Desc& d = descs[j & (C::DSLOTS - 1)];
-      if (d.b < 0) break;
-      const int kfirst = d.kfirst, ntiles = d.ntiles, split = d.split;
+      const bool last = !ok || d.b < 0;  // no item j: only the pending epilogue is left
+      const int ntiles = last ? 0 : d.ntiles;
+      bool acc_ok = ok;
+      float l_part[RH];  // bf16: this thread's part of item j's row sums
+#pragma unroll
+      for (int r = 0; r < RH; ++r) l_part[r] = 0.f;
+      const int kfirst = d.kfirst;
       const int lo_u = d.lo_u, hi_u = d.hi_u, lo_x = d.lo_x, hi_x = d.hi_x;
       uint8_t* sl = slot_of(j);
-      const long long* rows = reinterpret_cast<const long long*>(sl + C::SL_ROWS);
       const int2* rng = reinterpret_cast<const int2*>(sl + C::SL_RANGE);
       const float* sm_cs = reinterpret_cast<const float*>(sl + C::SL_CS);
       float2* sm_csm = reinterpret_cast<float2*>(sl + C::SL_CSM);
       float* sm_thr = reinterpret_cast<float*>(sl + C::SL_THR);
       float* sm_mraw = reinterpret_cast<float*>(sl + C::SL_MRAW);
-      const float* sm_sink = reinterpret_cast<const float*>(sl + C::SL_SINK);
-      float l_part[RH];  // bf16: this thread's part of the row sums
-#pragma unroll
-      for (int r = 0; r < RH; ++r) l_part[r] = 0.f;
       // O^T (and, FP8, the row sums) of this item accumulate in TMEM region
       // j & 1: bf16, 16 columns (r: P_hi, NT + r: P_lo), all read by every
       // thread; FP8, this group's 16 columns (hi terms of its rows, then lo).
       const uint32_t o_tm = tmem + lane_off + C::COL_O + (j & 1) * C::N2 + col_o;
       const uint32_t l_tm = tmem + lane_off + C::COL_L + (j & 1) * C::N2 + col_o;
-      // wait until the O^T MMAs of tile k have completed (all lanes agree)
-      auto wait_o = [&](int k) -> bool {
-        const bool ok_w = __all_sync(FULL, mbar_wait(&o_full[k & 1], (k >> 1) & 1, a.err));
-        if (ok_w) tmem_fence_after();
-        return ok_w;
-      };
-
-      bool acc_ok = true;
       for (int n = 0; n < ntiles; ++n, ++g) {
         const int bb = g & 1;
         bool ok_s = acc_ok && !*abort_flag;
@@ -958,183 +1156,24 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         tmem_fence_before();
         mbar_arrive(&p_ready[bb]);
         if (grp == 0 && i == 0) *tiles_done = g + 1;  // lets the scheduler draw more work
+        if (n == 0 && pend >= 0) {  // the previous item's epilogue
+          if (!epilogue(pend, pend_g, pend_nt, pend_ok, l_pend)) acc_ok = false;
+          pend = -1;
+        }
       }
       // the item's O^T (FP8: and row sums) once its last tile's MMAs are done
-      float acc[RH], lsum[RH];
-#pragma unroll
-      for (int r = 0; r < RH; ++r) {
-        acc[r] = 0.f;
-        lsum[r] = 0.f;
+      if (pend >= 0) {  // no tile of item j ran the pending epilogue (none, or the end)
+        if (!epilogue(pend, pend_g, pend_nt, pend_ok && ok, l_pend)) acc_ok = false;
+        pend = -1;
       }
-      if (__all_sync(FULL, acc_ok && ntiles > 0 && !*abort_flag)) {
-        acc_ok = wait_o(g - 1);
-        if (acc_ok) {
-          float o[16];
-          tmem_ld16_raw(o_tm, o);
-          if constexpr (C::BF16) {
+      if (last) break;
+      pend = j;
+      pend_g = g - 1;
+      pend_nt = ntiles;
+      pend_ok = acc_ok;
 #pragma unroll
-            for (int r = 0; r < RH; ++r) acc[r] = o[r] + o[NT + r];  // P = P_hi + P_lo
-          } else {
-#pragma unroll
-            for (int r = 0; r < RH; ++r) acc[r] = fmaf(o[RH + r], 0.0625f, o[r]);  // P_hi + (16 P_lo) / 16
-            tmem_ld16_raw(l_tm, o);
-#pragma unroll
-            for (int r = 0; r < RH; ++r) lsum[r] = fmaf(o[RH + r], 0.0625f, o[r]);
-          }
-        }
-      }
-      tmem_fence_before();
-      mbar_arrive(&o_free[j & 1]);  // region j & 1 may take item j + 2
-      ok = named_bar_and(gbar, GT, acc_ok);
-      if (!ok) *abort_flag = 1;
-
-      // ---- epilogue: normaliser and LSE per row, then the O rows ----------
-      if constexpr (C::BF16) {
-        // row sums: over the lanes, then over the group's four warps
-#pragma unroll
-        for (int r = 0; r < RH; ++r) {
-          float v = l_part[r];
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-          l_part[r] = v;
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int r = 0; r < RH; ++r) lred[q4 * 32 + r0 + r] = l_part[r];
-        }
-        named_bar(gbar, GT);
-#pragma unroll
-        for (int r = 0; r < RH; ++r)
-          lsum[r] = lred[r0 + r] + lred[32 + r0 + r] + lred[64 + r0 + r] + lred[96 + r0 + r];
-      }
-      // Thread i < RH derives row r0 + i's normaliser and LSE (the row sum
-      // is in every thread: FP8 from TMEM, bf16 from the reduction above)
-      // and shares the normaliser through shared memory.
-      const bool failed = !ok;
-      float* sm_inv = reinterpret_cast<float*>(smem + C::OFF_INV);
-      if (i < RH) {
-        float lt = 0.f;
-#pragma unroll
-        for (int r = 0; r < RH; ++r)
-          if (r == i) lt = lsum[r];
-        const int rr = r0 + i;
-        const long long row = rows[rr];
-        // attention sink of the row's head (one split only; with splits the
-        // merge adds it): one more exp2(sink) term in the denominator
-        const float sink = a.num_splits == 1 ? sm_sink[rr] : -INFINITY;
-        float inv = 0.f, res = failed ? -INFINITY : sink;
-        if (lt > 0.f && !failed) {
-          const float m = -sm_csm[rr].y;
-          float mref = m, l2 = lt, scl = 1.f;
-          if (sink != -INFINITY) {
-            const float sl = sink * kLog2e;
-            mref = fmaxf(m, sl);
-            scl = fast_exp2(m - mref);
-            l2 = fmaf(lt, scl, fast_exp2(sl - mref));
-          }
-          inv = a.v_scale * scl / l2;
-          res = (mref + log2f(l2)) * kLn2;
-        }
-        sm_inv[rr] = inv;
-        if (row >= 0) {
-          if (a.num_splits == 1) {
-            if (a.lse) a.lse[row] = res;
-          } else {
-            a.lse_part[(long long)split * rows_total + row] = res;
-          }
-        }
-      }
-      named_bar(gbar, GT);
-      float* dst = a.num_splits == 1 ? a.out : a.o_part + (long long)split * rows_total * C::D;
-#pragma unroll
-      for (int r = 0; r < RH; ++r) {
-        const long long row = rows[r0 + r];
-        if (row >= 0) dst[row * C::D + i] = acc[r] * sm_inv[r0 + r];
-      }
-
-      // ---- fused merge (PDA_FLAG_FUSED_MERGE): the split that arrives last
-      // for these rows combines every split's partials by log-sum-exp; each
-      // row group counts and merges its own rows --------------------------
-      if (a.num_splits > 1 && a.fused_merge) {
-        __threadfence();  // this split's partials are visible device-wide ...
-        named_bar(gbar, GT);  // (and every sm_inv read is done: sm_lse reuses it)
-        if (i == 0) {     // ... before the group counts itself in
-          int* ctr = a.merge_ctr +
-                     (((long long)d.b * a.Hkv + d.kvh) * a.row_tiles + d.rt) * kMergeCtrPerGroup + grp;
-          merge_flag[grp] = atomicAdd(ctr, 1) == a.num_splits - 1;
-        }
-        named_bar(gbar, GT);
-        if (merge_flag[grp]) {
-          __threadfence();
-          const int S = a.num_splits;  // <= 128
-          // (1) per row: lse = m + ln sum_s exp(lse_s - m); warp q4 takes the
-          // group's rows q4, q4 + 4, ...; lane l holds splits l, l + 32, l + 64, l + 96.
-          constexpr int RW = (RH + 3) / 4;
-          float v[RW][4];
-#pragma unroll
-          for (int k = 0; k < RW; ++k) {
-            const int rr = q4 + 4 * k;
-            const long long row = rr < RH ? rows[r0 + rr] : -1;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int spl = c * 32 + lane;
-              v[k][c] = row >= 0 && spl < S ? __ldcg(a.lse_part + (long long)spl * rows_total + row)
-                                            : -INFINITY;
-            }
-          }
-#pragma unroll
-          for (int k = 0; k < RW; ++k) {
-            // the row's attention sink is one more part: lse = sink, o = 0
-            const int rr = q4 + 4 * k;
-            const long long rrow = rr < RH ? rows[r0 + rr] : -1;
-            const float sink = rrow >= 0 ? sm_sink[r0 + rr] : -INFINITY;
-            float m = fmaxf(fmaxf(v[k][0], v[k][1]), fmaxf(v[k][2], v[k][3]));
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-            m = fmaxf(m, sink);
-            float sum = 0.f;
-            if (m != -INFINITY) {
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                if (v[k][c] != -INFINITY) sum += fast_exp2((v[k][c] - m) * kLog2e);
-              if (lane == 0 && sink != -INFINITY) sum += fast_exp2((sink - m) * kLog2e);
-            }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
-            if (lane == 0 && rr < RH) sm_lse[r0 + rr] = m == -INFINITY ? -INFINITY : m + log2f(sum) * kLn2;
-          }
-          named_bar(gbar, GT);
-          // (2) out[row, i] = sum_s exp(lse_s - lse) * o_s[row, i] over this
-          // thread's rows; the rows' loads of one split go out together
-#pragma unroll
-          for (int r = 0; r < RH; ++r) acc[r] = 0.f;
-          for (int spl = 0; spl < S; ++spl) {
-            float ls[RH], ov[RH];
-#pragma unroll
-            for (int r = 0; r < RH; ++r) {
-              const long long row = rows[r0 + r];
-              const long long idx = (long long)spl * rows_total + (row >= 0 ? row : 0);
-              ls[r] = row >= 0 ? __ldcg(a.lse_part + idx) : -INFINITY;
-              ov[r] = row >= 0 ? __ldcg(a.o_part + idx * C::D + i) : 0.f;
-            }
-#pragma unroll
-            for (int r = 0; r < RH; ++r)
-              if (ls[r] != -INFINITY)
-                acc[r] = fmaf(fast_exp2((ls[r] - sm_lse[r0 + r]) * kLog2e), ov[r], acc[r]);
-          }
-#pragma unroll
-          for (int r = 0; r < RH; ++r) {
-            const long long row = rows[r0 + r];
-            if (row >= 0) a.out[row * C::D + i] = acc[r];
-          }
-          if (i < RH && rows[r0 + i] >= 0 && a.lse) a.lse[rows[r0 + i]] = sm_lse[r0 + i];
-        }
-      }
-      named_bar(gbar, GT);  // the group no longer reads item j's state and descriptor
-      if (i == 0) {
-        mbar_arrive(&st_free[j & 1]);
-        mbar_arrive(&desc_free[j & (C::DSLOTS - 1)]);
-      }
+      for (int r = 0; r < RH; ++r) l_pend[r] = l_part[r];
+      acc_prev = acc_ok;
     }
     if (!ok) *abort_flag = 1;
   }
