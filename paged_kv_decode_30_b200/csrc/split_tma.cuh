@@ -1040,11 +1040,16 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           const float4 t = reinterpret_cast<const float4*>(sm_thr + r0)[r / 4];
           want = want | (s[r] > t.x) | (s[r + 1] > t.y) | (s[r + 2] > t.z) | (s[r + 3] > t.w);
         }
-        // one group barrier decides for the tile (and propagates failures)
-        const bool flag = named_bar_or_and(gbar, GT, want, ok_s, &ok_s);
-        if (!ok_s) {
-          acc_ok = false;
-          break;
+        // One group barrier decides for the tile: a failed wait counts as a
+        // want, and only then (rarely) do the OR of the wants and the AND of
+        // the waits' outcomes follow separately.
+        bool flag = false;
+        if (named_bar_or(gbar, GT, want || !ok_s)) {
+          flag = named_bar_or_and(gbar, GT, want, ok_s, &ok_s);
+          if (!ok_s) {
+            acc_ok = false;
+            break;
+          }
         }
         if (flag) {
 #pragma unroll
