@@ -1121,7 +1121,9 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         // them every tile also keeps this warp's o_full phases in step, so
         // the o_full(g - 1) waits above and after the loop never see a phase
         // that is two behind.
-        if (g >= 2 && !wait_o(g - 2)) acc_ok = false;
+        // (Each lane waits for itself: no TMEM access follows, and a lane whose
+        // wait fails clears acc_ok, which the next group barrier spreads.)
+        if (g >= 2 && !mbar_wait(&o_full[g & 1], ((g - 2) >> 1) & 1, a.err)) acc_ok = false;
         // P^T row of token i (row-major over the N2 columns, swizzled chunks)
         uint8_t* sp = smem + C::OFF_P + bb * C::P_BUF + (i >> 3) * C::P_SBO + (i & 7) * C::P_ROW;
         const int pswz = C::P_ROW == 64 ? ((i & 7) >> 1) & 3 : ((i & 7) >> 2) & 1;
