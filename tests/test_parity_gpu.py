@@ -341,3 +341,56 @@ def test_full_size_fp8_verify_native_qk(lib):
     seqs = [0, 17, 63]
     ref_out, ref_lse = U.run_oracle(inp, seqs=seqs, native_qk=True)
     U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, FP8, "fp8 verify native qk")
+
+
+def _visible_tiles(wl, L, tile=128):
+    """128-token tiles of the union of a sequence's rows' visible key ranges
+    (readings R2, R3): the first query row's start to the last row's end."""
+    W_ = wl.window
+
+    def rng(i):
+        if wl.causal_offset == B.PDA_CAUSAL_OFF:
+            pos, hi = L - 1, L
+        else:
+            pos = (L - wl.q_len + i) if wl.causal_offset == B.PDA_CAUSAL_BOTTOM_RIGHT else wl.causal_offset + i
+            hi = min(L, pos + 1)
+        lo = max(0, pos - W_ + 1) if W_ > 0 else 0
+        return lo, hi
+
+    lo, _ = rng(0)
+    _, hi = rng(wl.q_len - 1)
+    return (hi + tile - 1) // tile - lo // tile if hi > lo else 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [W.VARLEN, W.FP8_VERIFY], ids=lambda w: w.name)
+def test_work_queue_hands_out_longest_sequences_first(lib, wl):
+    """The tensor-core kernel's prologue writes the queue order into the
+    workspace after the counter header: a permutation of the sequences with
+    their visible 128-token tiles non-increasing."""
+    import torch
+    inp = W.generate(wl, device="cuda")
+    flags = B.PDA_FLAG_TENSOR_CORES
+    params = B.make_params(
+        batch=wl.batch, q_len=wl.q_len, num_q_heads=wl.num_q_heads,
+        num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, page_size=wl.page_size,
+        max_pages_per_seq=inp["page_table"].shape[1], num_pages=inp["k_pages"].shape[0],
+        scale=W.scale_of(wl), causal_offset=wl.causal_offset, window=wl.window,
+        kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"], num_splits=1, flags=flags)
+    assert B.plan_kernel(params) == B.PDA_KERNEL_SPLIT_TMA
+    ws = torch.full((B.workspace_bytes(params),), 0xAB, dtype=torch.uint8, device="cuda")
+    B.paged_decode_attn(inp["q"], inp["k_pages"], inp["v_pages"], inp["page_table"],
+                        inp["kv_lens"], num_kv_heads=wl.num_kv_heads, scale=W.scale_of(wl),
+                        causal_offset=wl.causal_offset, window=wl.window,
+                        kv_scale=inp["kv_scale"], num_splits=1, flags=flags, workspace=ws)
+    torch.cuda.synchronize()
+    M = wl.q_len * (wl.num_q_heads // wl.num_kv_heads)
+    assert M <= 32  # one row tile per (sequence, kv head) at these shapes
+    header = 64 + wl.batch * wl.num_kv_heads * 1 * 4 * 4
+    off = (header + 255) // 256 * 256
+    order = ws[off:off + 4 * wl.batch].cpu().view(torch.int32).tolist()
+    assert sorted(order) == list(range(wl.batch))
+    lens = inp["kv_lens"].cpu().tolist()
+    tiles = [_visible_tiles(wl, lens[b]) for b in order]
+    assert all(tiles[k] >= tiles[k + 1] for k in range(len(tiles) - 1)), tiles
+    assert tiles[0] > tiles[-1]  # the workloads mix lengths: the order is not trivial
