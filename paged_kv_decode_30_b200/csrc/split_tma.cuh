@@ -196,10 +196,6 @@ __device__ __forceinline__ void tmem_ld16_raw(uint32_t taddr, float* v) {
   float (&vv)[16] = *reinterpret_cast<float(*)[16]>(v);
   tmem_ld16(taddr, vv);
 }
-__device__ __forceinline__ void tmem_ld32_raw(uint32_t taddr, float* v) {
-  float (&vv)[32] = *reinterpret_cast<float(*)[32]>(v);
-  tmem_ld32(taddr, vv);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

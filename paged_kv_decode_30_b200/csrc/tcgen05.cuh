@@ -11,7 +11,6 @@
 
 namespace pda {
 
-
 // Shared-memory matrix descriptor: start address, leading- and stride-
 // dimension byte offsets, and the swizzle mode of the canonical layout.
 // Swizzled atoms are 8 rows of 128 (SW128), 64 (SW64) or 32 (SW32) bytes
@@ -42,17 +41,6 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16: f16 A and B, fp32 D.
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
-  return (1u << 4)                              // D format: f32
-         | (0u << 7) | (0u << 10)               // A, B format: f16
-         | ((a_mn_major ? 1u : 0u) << 15)
-         | ((b_mn_major ? 1u : 0u) << 16)
-         | ((uint32_t)(N >> 3) << 17)
-         | ((uint32_t)(M >> 4) << 24);
-}
-
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -74,26 +62,6 @@ __device__ __forceinline__ void tmem_fence_before() {
 }
 __device__ __forceinline__ void tmem_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 32 consecutive fp32 TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
 // 16 consecutive fp32 TMEM columns of this thread's lane.
@@ -124,49 +92,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
       : "memory");
 #pragma unroll
   for (int k = 0; k < 8; ++k) v[k] = __uint_as_float(r[k]);
-}
-
-// Two runs of 16 fp32 columns (at ta and tb) of this thread's lane, one wait.
-__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float* va, float* vb) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(ta), "r"(tb)
-      : "memory");
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    va[k] = __uint_as_float(r[k]);
-    vb[k] = __uint_as_float(r[16 + k]);
-  }
-}
-
-// Two runs of 8 fp32 columns (at ta and tb) of this thread's lane, one wait.
-__device__ __forceinline__ void tmem_ld8x2(uint32_t ta, uint32_t tb, float* va, float* vb) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%16];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%17];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(ta), "r"(tb)
-      : "memory");
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    va[k] = __uint_as_float(r[k]);
-    vb[k] = __uint_as_float(r[8 + k]);
-  }
 }
 
 // Store 16 (or 8) fp32 values to consecutive TMEM columns of this thread's
@@ -249,28 +174,6 @@ __device__ __forceinline__ bool named_bar_or_and(int id, int threads, bool want,
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
                : "memory");
-}
-
-// 8 e4m3 codes -> 8 f16 packed as a uint4 (exact).
-__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint2 u) {
-  uint4 o;
-  uint32_t* w = reinterpret_cast<uint32_t*>(&o);
-  const uint32_t in[2] = {u.x, u.y};
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
-          static_cast<__nv_fp8x2_storage_t>((in[k] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
-      w[2 * k + h] = (uint32_t)hr.x | ((uint32_t)hr.y << 16);
-    }
-  }
-  return o;
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 }  // namespace pda
