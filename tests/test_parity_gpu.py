@@ -70,6 +70,15 @@ CASES = [
     wl("tc_fp8_fixed_offset_empty", batch=3, q_len=4, num_q_heads=64, num_kv_heads=8,
        head_dim=128, page_size=128, kv_dtype=FP8, causal_offset=40, window=30,
        kv_lens=("fixed", [0, 20, 700]), extra_pages=2),
+    # FP8 tensor-core path with peaked scores: 1% of the keys scaled by 8 and a
+    # large softmax scale, so the weights span many binades and most fall far
+    # below the largest (the two-term e4m3 P and the lazy max rescale)
+    wl("tc_fp8_peaked_g8_q4", batch=2, q_len=4, num_q_heads=32, num_kv_heads=4, head_dim=128,
+       page_size=128, kv_dtype=FP8, scale=0.25, causal_offset=BR, peaked_frac=0.01,
+       kv_lens=("fixed", [3000, 5000])),
+    # the bf16 tensor-core path (4 packed rows) on the same kind of scores
+    wl("tc_bf16_peaked_g4", batch=2, num_q_heads=16, num_kv_heads=4, head_dim=128,
+       page_size=16, scale=0.25, peaked_frac=0.01, kv_lens=("fixed", [3000, 8000])),
 ]
 
 
