@@ -974,14 +974,12 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       // j & 1: bf16, 16 columns (r: P_hi, NT + r: P_lo), all read by every
       // thread; FP8, this group's 16 columns (hi terms of its rows, then lo).
       const uint32_t o_tm = tmem + lane_off + C::COL_O + (j & 1) * C::N2 + col_o;
-      // this thread's rows' lazy-rescale thresholds and {scale, -m}, kept in
-      // registers and reloaded whenever a tile moves the max
-      float4 thr4[RH / 4], csm4[RH / 2];
+      // this thread's rows' lazy-rescale thresholds, kept in registers and
+      // reloaded whenever a tile moves the max
+      float4 thr4[RH / 4];
       auto load_row_consts = [&]() {
 #pragma unroll
         for (int k = 0; k < RH / 4; ++k) thr4[k] = reinterpret_cast<const float4*>(sm_thr + r0)[k];
-#pragma unroll
-        for (int k = 0; k < RH / 2; ++k) csm4[k] = reinterpret_cast<const float4*>(sm_csm + r0)[k];
       };
       load_row_consts();
       const uint32_t l_tm = tmem + lane_off + C::COL_L + (j & 1) * C::N2 + col_o;
@@ -1116,7 +1114,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         float* p = s;
 #pragma unroll
         for (int r = 0; r < RH; r += 2) {
-          const float4 c = csm4[r / 2];
+          const float4 c = reinterpret_cast<const float4*>(sm_csm + r0)[r / 2];
           p[r] = fast_exp2(fmaf(s[r], c.x, c.y));
           p[r + 1] = fast_exp2(fmaf(s[r + 1], c.z, c.w));
           if constexpr (C::BF16) {
