@@ -151,6 +151,26 @@ def test_split_planner(lib):
     assert B.choose_num_splits(win, 148) <= 256 // 16
 
 
+def test_split_planner_persistent_kernel(lib):
+    """The persistent tensor-core kernel takes no split once there are 1.5
+    (sequence, kv head, row tile) units per SM (its queue hands out the longest
+    sequences first); fewer units keep the wave model, as does the CUDA-core
+    kernel."""
+    def p(batch, **kw):
+        return headline_params(batch=batch, num_q_heads=4, num_kv_heads=1, max_kv_len=65536,
+                               max_pages_per_seq=4096, **kw)
+    assert B.plan_kernel(p(222)) == B.PDA_KERNEL_SPLIT_TMA
+    assert B.choose_num_splits(p(222), 148) == 1      # 2 * 222 = 3 * 148
+    assert B.choose_num_splits(p(221), 148) > 1       # below: the wave model splits
+    assert B.choose_num_splits(p(222, flags=B.PDA_FLAG_CUDA_CORES), 148) > 1
+    fp8_verify = B.make_params(batch=64, q_len=4, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                               page_size=128, max_pages_per_seq=256, num_pages=16384,
+                               scale=0.08838834764831845, kv_dtype=B.PDA_KV_FP8_E4M3,
+                               kv_scale=0.01, causal_offset=B.PDA_CAUSAL_BOTTOM_RIGHT, window=4096)
+    assert B.plan_kernel(fp8_verify) == B.PDA_KERNEL_SPLIT_TMA
+    assert B.choose_num_splits(fp8_verify, 148) == 1
+
+
 def test_workspace_bytes(lib):
     rows = 128 * 32
     expect_o = 4 * rows * 128 * 4
