@@ -403,3 +403,35 @@ def test_work_queue_hands_out_longest_sequences_first(lib, wl):
     tiles = [_visible_tiles(wl, lens[b]) for b in order]
     assert all(tiles[k] >= tiles[k + 1] for k in range(len(tiles) - 1)), tiles
     assert tiles[0] > tiles[-1]  # the workloads mix lengths: the order is not trivial
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("flags", [B.PDA_FLAG_TENSOR_CORES, B.PDA_FLAG_CUDA_CORES],
+                         ids=["tensor_cores", "cuda_cores"])
+def test_fp8_value_decode_is_exact(lib, flags):
+    """Every e4m3 code through the whole path, bit for bit: each sequence sees
+    one key, so its weight is exactly 1 and out = fp32(decode(v) * kv_scale);
+    the V row of sequence b holds codes 128 b .. 128 b + 127 (NaN codes give
+    NaN)."""
+    import torch
+    Bn, Hq, Hkv, D, P = 2, 16, 1, 128, 16  # 16 packed rows: the FP8 tensor-core path
+    g = torch.Generator().manual_seed(7)
+    q = torch.randn(Bn, 1, Hq, D, generator=g).to(torch.bfloat16)
+    k_pages = torch.randint(0, 0x7E, (Bn, Hkv, P, D), generator=g, dtype=torch.uint8)
+    v_pages = torch.randint(0, 0x7E, (Bn, Hkv, P, D), generator=g, dtype=torch.uint8)
+    for b in range(Bn):
+        v_pages[b, 0, 0] = torch.arange(128 * b, 128 * b + 128, dtype=torch.int32).to(torch.uint8)
+    page_table = torch.arange(Bn, dtype=torch.int32).reshape(Bn, 1)
+    kv_lens = torch.ones(Bn, dtype=torch.int32)
+    kv_scale = 0.0371
+    out, lse, _ = B.paged_decode_attn(q.cuda(), k_pages.cuda(), v_pages.cuda(), page_table.cuda(),
+                                      kv_lens.cuda(), num_kv_heads=Hkv, scale=D ** -0.5,
+                                      kv_scale=kv_scale, num_splits=1, flags=flags)
+    torch.cuda.synchronize()
+    assert B.last_device_error() == 0
+    dec = v_pages[:, 0, 0].view(torch.float8_e4m3fn).float()          # [B, D], exact
+    want = (dec * torch.tensor(kv_scale, dtype=torch.float32))[:, None, None, :].expand(Bn, 1, Hq, D)
+    got = out.cpu()
+    assert torch.equal(torch.isnan(got), torch.isnan(want))
+    fin = ~torch.isnan(want)
+    assert torch.equal(got[fin], want[fin]), (got[fin] - want[fin]).abs().max()
