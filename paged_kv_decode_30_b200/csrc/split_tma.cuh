@@ -12,11 +12,14 @@
 // Work item: the packed rows (NT of them) of one (sequence, kv head, split,
 // row tile); a CTA runs items one after another, a 128-token tile at a time
 // (the MMA M dimension): S^T = K Q^T, then O^T = V^T P^T. One CTA per SM;
-// the grid is min(items, SMs) and items come from an atomic counter, so
-// SMs that finish short sequences take the next item at once.
+// the grid is min(items, SMs) and items come from an atomic counter, in the
+// order a prologue kernel sets (longest sequences first; it also zeroes the
+// counters and writes the FP8 Q operands), so SMs that finish short items
+// take the next one at once and the CTAs finish close together.
 //  * warp 7 (scheduler): draws items, computes their key ranges and the page
 //    ids of their first tiles into a 4-deep descriptor ring, and writes each
-//    item's Q operand and per-row state (one item ahead of the MMAs).
+//    item's Q operand (bf16: a swizzled copy; FP8: one bulk copy of the
+//    prologue's image) and per-row state, one item ahead of the MMAs.
 //  * warp 0 (producer): TMA loads of each page segment of the K and V tiles
 //    into a STAGES-deep ring in the canonical 128B-swizzled UMMA layout (one
 //    tensor map per pool: rows = (page, kv head, token), 128 elements per
@@ -30,7 +33,9 @@
 //      FP8 K/V: S^T with kind::f8f6f4 straight from the e4m3 K stage, B =
 //        [Q_hi; Q_lo], an exact two-term e4m3 split of each bf16 q row
 //        scaled by a power of two; O^T with kind::f8f6f4 straight from the
-//        e4m3 V stage (MN-major), B = P^T as two e4m3 terms [P_hi; 16 P_lo].
+//        e4m3 V stage (MN-major), B = P^T as two e4m3 terms [P_hi; 16 P_lo];
+//        and the row sums of P^T (the normaliser) as the same B against a
+//        tile of e4m3 ones.
 //  * warps 3-6 (and, FP8, 8-19 by item rows: groups of four warps with 8
 //    rows each) (softmax): thread i = TMEM lane i = token i of S^T and
 //    head-dim element i of O^T. p = exp2(s * c - m) in fp32 with a lazily
@@ -38,8 +43,9 @@
 //    the item's tiles; a tile that moves the max rescales it in place first.
 //    On tiles with keys that no row may see they also zero those keys' V
 //    rows in the stage, so NaN bytes never meet a zero weight in the MMA.
-//    After an item: normalise and store O and the LSE (or the split's
-//    partials; the split that arrives last for its rows merges them all).
+//    An item's epilogue (normalise, store O and the LSE, or the split's
+//    partials; with the fused merge, the split that arrives last for its
+//    rows merges them all) runs after the next item's first tile.
 //  * Every wait is bounded; group exits go through bar.red.and.
 #pragma once
 
@@ -944,7 +950,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     int g = 0;  // tiles of this CTA so far (over all items)
     bool ok = true, acc_prev = true;
     // the item whose epilogue is pending (-1: none), its last tile, tile
-    // count, status and (bf16) partial row sums
+    // count, status and partial row sums (bf16; FP8 sums by MMA)
     int pend = -1, pend_g = 0, pend_nt = 0;
     bool pend_ok = true;
     float l_pend[RH];
