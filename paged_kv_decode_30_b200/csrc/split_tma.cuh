@@ -216,6 +216,22 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
   return r;
 }
 
+// Two weights -> their two-term e4m3 split, low byte first: returns
+// e4m3(p) in the low 16 bits and e4m3(16 (p - e4m3(p))) in the high 16.
+// Done in f16x2: p (<= 2^8) rounds to f16 first; p16 - hi is then exact in
+// f16 (hi is p16 on e4m3's coarser grid) and so is the factor 16, so the
+// pair keeps about 8 significant bits of p.
+__device__ __forceinline__ uint32_t e4m3_split2(float p0, float p1) {
+  const __half2 a = __floats2half2_rn(p0, p1);
+  const __nv_fp8x2_storage_t h =
+      __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(a), __NV_SATFINITE, __NV_E4M3);
+  const __half2 d = static_cast<__half2>(__nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3));
+  const __half2 l = __hmul2(__hsub2(a, d), __float2half2_rn(16.f));
+  const __nv_fp8x2_storage_t lo =
+      __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(l), __NV_SATFINITE, __NV_E4M3);
+  return (uint32_t)h | ((uint32_t)lo << 16);
+}
+
 // Two e4m3 codes (low byte first) -> two floats, exactly.
 __device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t codes) {
   const __half2_raw hr =
@@ -1044,18 +1060,24 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         // thr = (m + kRescaleLog2) / cs (-inf until the row's first finite
         // score), so it is one compare per score.
         constexpr float kRescaleLog2 = 8.f;
-        bool want = false;
+        auto wants = [&]() {
+          bool w = false;
 #pragma unroll
-        for (int r = 0; r < RH; r += 4) {
-          const float4 t = thr4[r / 4];
-          want = want | (s[r] > t.x) | (s[r + 1] > t.y) | (s[r + 2] > t.z) | (s[r + 3] > t.w);
-        }
+          for (int r = 0; r < RH; r += 4) {
+            const float4 t = thr4[r / 4];
+            w = w | (s[r] > t.x) | (s[r + 1] > t.y) | (s[r + 2] > t.z) | (s[r + 3] > t.w);
+          }
+          return w;
+        };
         // One group barrier decides for the tile: a failed wait counts as a
         // want, and only then (rarely) do the OR of the wants and the AND of
         // the waits' outcomes follow separately.
+        bool any;
+        if constexpr (!C::BF16) any = named_bar_any_gt8(gbar, GT, s, thr4[0], thr4[1], !ok_s);
+        else any = named_bar_or(gbar, GT, wants() || !ok_s);
         bool flag = false;
-        if (named_bar_or(gbar, GT, want || !ok_s)) {
-          flag = named_bar_or_and(gbar, GT, want, ok_s, &ok_s);
+        if (any) {
+          flag = named_bar_or_and(gbar, GT, wants(), ok_s, &ok_s);
           if (!ok_s) {
             acc_ok = false;
             break;
@@ -1161,12 +1183,10 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           uint32_t hi[2], lo[2];
 #pragma unroll
           for (int r = 0; r < RH; r += 4) {
-            const uint32_t h01 = f32x2_to_e4m3x2(p[r], p[r + 1]);
-            const uint32_t h23 = f32x2_to_e4m3x2(p[r + 2], p[r + 3]);
-            const float2 d01 = e4m3x2_to_f32x2(h01), d23 = e4m3x2_to_f32x2(h23);
-            hi[r / 4] = h01 | (h23 << 16);
-            lo[r / 4] = f32x2_to_e4m3x2(16.f * (p[r] - d01.x), 16.f * (p[r + 1] - d01.y)) |
-                        (f32x2_to_e4m3x2(16.f * (p[r + 2] - d23.x), 16.f * (p[r + 3] - d23.y)) << 16);
+            const uint32_t s01 = e4m3_split2(p[r], p[r + 1]);
+            const uint32_t s23 = e4m3_split2(p[r + 2], p[r + 3]);
+            hi[r / 4] = __byte_perm(s01, s23, 0x5410);  // the e4m3(p) halves
+            lo[r / 4] = __byte_perm(s01, s23, 0x7632);  // the residual halves
           }
           *reinterpret_cast<uint4*>(sp + ((grp ^ pswz) << 4)) = make_uint4(hi[0], hi[1], lo[0], lo[1]);
         }

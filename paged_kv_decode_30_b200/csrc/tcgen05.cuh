@@ -142,6 +142,32 @@ __device__ __forceinline__ bool named_bar_or(int id, int threads, bool v) {
   return r != 0;
 }
 
+// Lazy max test of eight scores fused with the group barrier: returns, in
+// every thread, the OR over the `threads` threads of (any s[k] > t[k]) or
+// `failed`. The compares chain through one predicate (setp with .or).
+__device__ __forceinline__ bool named_bar_any_gt8(int id, int threads, const float* s,
+                                                  float4 t0, float4 t1, bool failed) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "setp.gt.or.f32 p, %4, %12, p;\n\t"
+      "setp.gt.or.f32 p, %5, %13, p;\n\t"
+      "setp.gt.or.f32 p, %6, %14, p;\n\t"
+      "setp.gt.or.f32 p, %7, %15, p;\n\t"
+      "setp.gt.or.f32 p, %8, %16, p;\n\t"
+      "setp.gt.or.f32 p, %9, %17, p;\n\t"
+      "setp.gt.or.f32 p, %10, %18, p;\n\t"
+      "setp.gt.or.f32 p, %11, %19, p;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)failed), "r"(id), "r"(threads), "f"(s[0]), "f"(s[1]), "f"(s[2]),
+        "f"(s[3]), "f"(s[4]), "f"(s[5]), "f"(s[6]), "f"(s[7]), "f"(t0.x), "f"(t0.y),
+        "f"(t0.z), "f"(t0.w), "f"(t1.x), "f"(t1.y), "f"(t1.z), "f"(t1.w)
+      : "memory");
+  return r != 0;
+}
+
 // Named barrier over `threads` threads that also returns the AND of `v` over
 // them, so every thread takes the same branch afterwards.
 __device__ __forceinline__ bool named_bar_and(int id, int threads, bool v) {
