@@ -232,13 +232,6 @@ __device__ __forceinline__ uint32_t e4m3_split2(float p0, float p1) {
   return (uint32_t)h | ((uint32_t)lo << 16);
 }
 
-// Two e4m3 codes (low byte first) -> two floats, exactly.
-__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t codes) {
-  const __half2_raw hr =
-      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes & 0xFFFFu), __NV_E4M3);
-  return make_float2(__half2float(__ushort_as_half(hr.x)), __half2float(__ushort_as_half(hr.y)));
-}
-
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code & 0xFF), __NV_E4M3);
   return __half2float(*reinterpret_cast<const __half*>(&h));
