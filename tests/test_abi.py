@@ -84,6 +84,14 @@ def headline_params(**over):
     (dict(max_pages_per_seq=0), 1),
     (dict(num_splits=-1), 1),
     (dict(batch=-1), 1),
+    (dict(num_kv_heads=0), 1),
+    (dict(scale=-1.0), 1),
+    (dict(scale=float("inf")), 1),
+    (dict(kv_dtype=1, kv_scale=float("nan")), 1),
+    (dict(kv_dtype=1, kv_scale=float("inf")), 1),
+    (dict(max_kv_len=-1), 1),
+    (dict(max_pages_per_seq=1 << 27), 1),  # 2^27 pages x 16 tokens > INT_MAX
+    (dict(batch=65536), 2),
 ])
 def test_invalid_params_rejected_on_host(lib, over, status):
     p = headline_params(**over)
@@ -109,6 +117,18 @@ def test_misaligned_pointers(lib):
     assert st == 3
     st = lib.paged_decode_attn(ok, ok, ok, ok, ok, ctypes.byref(p), bad, ok, None)
     assert st == 3
+    # page table, kv_lens, lse and sinks need 4 bytes; the workspace 256
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    for args in ((ok, ok, ok, odd, ok, ok, ok), (ok, ok, ok, ok, odd, ok, ok),
+                 (ok, ok, ok, ok, ok, ok, odd)):
+        q, k, v, pt, kl, out, lse = args
+        assert lib.paged_decode_attn(q, k, v, pt, kl, ctypes.byref(p), out, lse, None) == 3
+    p.sinks = (1 << 20) + 2
+    assert lib.paged_decode_attn(ok, ok, ok, ok, ok, ctypes.byref(p), ok, ok, None) == 3
+    p = headline_params()
+    p.workspace = (1 << 20) + 16
+    p.workspace_bytes = 1 << 20
+    assert lib.paged_decode_attn(ok, ok, ok, ok, ok, ctypes.byref(p), ok, ok, None) == 3
 
 
 def test_empty_batch_is_a_no_op(lib):
