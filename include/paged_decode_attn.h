@@ -146,9 +146,10 @@ typedef struct {
  * counters: the work queue of its persistent CTAs and, per (sequence, kv
  * head, row tile) and softmax row group, how many splits have finished
  * (the last one merges).
- * The call zeroes that header itself (one small memset on `stream` before
- * the launch), so the workspace's contents before the call do not matter
- * and a call captured in a CUDA graph replays correctly. Every partial slot
+ * The tensor-core kernel's prologue (a small kernel launched on `stream`
+ * just before it) zeroes that header on every call, so the workspace's
+ * contents before the call do not matter and a call captured in a CUDA graph
+ * replays correctly. Every partial slot
  * a kernel reads was written earlier in the same call. If params->workspace is NULL the library
  * uses a grow-only buffer it owns, one per device, shared by every call on
  * that device: calls that may overlap on different streams must pass their

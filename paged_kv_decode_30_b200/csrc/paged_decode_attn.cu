@@ -182,8 +182,9 @@ int choose_splits(const pda_params* p, const Plan& pl, int num_sms) {
 
 // Workspace layout. The tensor-core kernel keeps its work-queue counter and
 // split-arrival counters per (sequence, kv head, row tile) at the front
-// (zeroed by a memset on the call's stream before the launch); the split
-// partials follow (o_part then lse_part).
+// (zeroed on every call by the kernel's prologue, launched just before it on
+// the call's stream), then the queue order and the FP8 Q operand images; the
+// split partials follow (o_part then lse_part).
 struct WsLayout {
   size_t counters;  // bytes of the counter header (0 for the FMA kernel)
   size_t order_off, qops_off;  // tensor-core kernel: queue order, FP8 Q images
