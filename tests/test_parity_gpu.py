@@ -275,7 +275,7 @@ def test_workspace_contents_do_not_matter(lib, case):
 
 def test_cuda_graph_replays(lib):
     """A call captured in a CUDA graph replays correctly many times (the
-    counter memset is part of the captured work)."""
+    prologue kernel that zeroes the counters is part of the captured work)."""
     case = [c for c in CASES if c.name.startswith("tc_fp8")][0]
     inp = W.generate(case)
     ref_out, ref_lse = U.run_oracle(inp)
