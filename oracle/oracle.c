@@ -33,6 +33,17 @@
  *  R5 KV pool layout is [num_pages, Hkv, page_size, D].
  *  R6 FP8 value = decode_e4m3(byte) * kv_scale, one scale for K and V.
  *  R8 a row that sees no key has out = 0 and lse = -inf.
+ *  R22 NVFP4 KV ("b12x 0.30.0, Kernel inventory": NVFP4 float4_e2m1fn with
+ *      E4M3 scales per 16 elements, "BF16-to-FP4 TMA quantization" row:
+ *      packed NVFP4 plus scale tiles): element d of a token row is the
+ *      E2M1 nibble d % 2 (low nibble first) of byte d / 2 of the code pool
+ *      [num_pages, Hkv, P, D/2]; each block of 16 consecutive elements of
+ *      the row has one E4M3 scale in the scale pool [num_pages, Hkv, P,
+ *      D/16]; value = e2m1(code) * e4m3(block scale) * kv_scale.
+ *  R23 NVFP4 quantisation of new K/V rows (the cache producer's rule): per
+ *      block of 16 elements, in single precision with nearest-even rounding
+ *      and saturation, q = x / kv_scale, scale = e4m3(max |q| / 6), code =
+ *      e2m1(q / scale); a block whose scale is zero stores +0 codes.
  *  R18 the attention-sink bias of query head h is a logit sink[h] (natural
  *      log units, same scale as scale * q.k) that adds exp(sink[h]) to the
  *      softmax denominator and contributes no value: out = sum_j
@@ -42,8 +53,10 @@
  * Pins (tests/test_oracle.py): brute-force dense attention over the unpaged
  * K/V, page-permutation invariance, split-merge invariance, closed forms
  * (equal keys -> mean of V, one key -> v, one-hot V -> probabilities),
- * e4m3/bf16 decode against torch's independent float8/bfloat16 casts, and
- * hand-derived golden fixtures.
+ * e4m3/bf16 decode against torch's independent float8/bfloat16 casts,
+ * e2m1 decode and encode against ml_dtypes' float4_e2m1fn (another
+ * independent implementation) and hand-worked codes, and hand-derived
+ * golden fixtures.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -fPIC -shared oracle.c -o liboracle.so -lm
  */
@@ -60,6 +73,7 @@
 
 #define ORACLE_KV_BF16 0
 #define ORACLE_KV_FP8_E4M3 1
+#define ORACLE_KV_NVFP4 2
 
 #define ORACLE_CAUSAL_OFF (-1)
 #define ORACLE_CAUSAL_BOTTOM_RIGHT (-2)
@@ -89,12 +103,34 @@ double oracle_e4m3_to_double(uint8_t code) {
   return s ? -mag : mag;
 }
 
-/* One K or V element of the pool, decoded to double. */
-static double kv_elem(const void* pool, int kv_dtype, double kv_scale,
-                      int64_t index) {
+/* FP4 E2M1 from its fields: sign bit, 2 exponent bits with bias 1, 1
+ * mantissa bit. exponent 0 is subnormal: m/2 * 2^(1-1); every other code is
+ * (1 + m/2) * 2^(e-1). No infinities or NaN; largest magnitude 6. */
+double oracle_e2m1_to_double(uint8_t code) {
+  int s = (code >> 3) & 1;
+  int e = (code >> 1) & 0x3;
+  int m = code & 0x1;
+  double mag;
+  if (e == 0)
+    mag = (double)m / 2.0;
+  else
+    mag = ldexp(1.0 + (double)m / 2.0, e - 1);
+  return s ? -mag : mag;
+}
+
+/* One K or V element of the pool, decoded to double. `index` counts
+ * elements of [num_pages, Hkv, P, D]; for NVFP4 (reading R22) the codes sit
+ * two per byte and `scales` holds one E4M3 code per 16 elements. */
+static double kv_elem(const void* pool, const void* scales, int kv_dtype,
+                      double kv_scale, int64_t index) {
   if (kv_dtype == ORACLE_KV_BF16)
     return oracle_bf16_to_double(((const uint16_t*)pool)[index]);
-  return oracle_e4m3_to_double(((const uint8_t*)pool)[index]) * kv_scale;
+  if (kv_dtype == ORACLE_KV_FP8_E4M3)
+    return oracle_e4m3_to_double(((const uint8_t*)pool)[index]) * kv_scale;
+  const uint8_t byte = ((const uint8_t*)pool)[index / 2];
+  const uint8_t code = (index % 2) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+  const double block = oracle_e4m3_to_double(((const uint8_t*)scales)[index / 16]);
+  return oracle_e2m1_to_double(code) * block * kv_scale;
 }
 
 /* Position of query row i of sequence b (reading R2/R3). */
@@ -122,8 +158,10 @@ static int check_args(const int32_t* kv_lens, int B, int q_len, int Hq, int Hkv,
   if (B < 0 || q_len < 1 || Hq < 1 || Hkv < 1 || D < 1 || page_size < 1 ||
       max_pages < 0 || num_pages < 0 || Hq % Hkv != 0)
     return ORACLE_BAD_ARG;
-  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3)
+  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3 &&
+      kv_dtype != ORACLE_KV_NVFP4)
     return ORACLE_BAD_ARG;
+  if (kv_dtype == ORACLE_KV_NVFP4 && D % 16 != 0) return ORACLE_BAD_ARG;
   if (causal_offset < ORACLE_CAUSAL_BOTTOM_RIGHT) return ORACLE_BAD_ARG;
   *max_len = 0;
   for (int b = 0; b < B; ++b) {
@@ -142,6 +180,7 @@ static int check_args(const int32_t* kv_lens, int B, int q_len, int Hq, int Hkv,
  * with no value vector (reading R18).
  */
 static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_pages,
+                      const void* k_scales, const void* v_scales,
                       const int32_t* page_table, const int32_t* kv_lens, int q_len,
                       int Hq, int Hkv, int D, int page_size, int max_pages,
                       int num_pages, float scale, int causal_offset, int window,
@@ -176,7 +215,7 @@ static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_page
     double dot = 0.0;
     for (int d = 0; d < D; ++d)
       dot += oracle_bf16_to_double(qrow[d]) *
-             kv_elem(k_pages, kv_dtype, dkv_scale, base + d);
+             kv_elem(k_pages, k_scales, kv_dtype, dkv_scale, base + d);
     s[j] = dscale * dot;
     if (s[j] > m) m = s[j];
     ++nvis;
@@ -206,7 +245,7 @@ static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_page
     const int64_t row = j % page_size;
     const int64_t base = (((int64_t)page * Hkv + g) * page_size + row) * D;
     for (int d = 0; d < D; ++d)
-      orow[d] += p * kv_elem(v_pages, kv_dtype, dkv_scale, base + d);
+      orow[d] += p * kv_elem(v_pages, v_scales, kv_dtype, dkv_scale, base + d);
   }
   return ORACLE_OK;
 }
@@ -217,13 +256,17 @@ static int oracle_row(const uint16_t* q, const void* k_pages, const void* v_page
  * the tests build split partials from the same definition.
  *
  * q          bf16 bits  [B, q_len, Hq, D]
- * k/v_pages  bf16 bits or e4m3 bytes  [num_pages, Hkv, page_size, D]
+ * k/v_pages  bf16 bits or e4m3 bytes  [num_pages, Hkv, page_size, D], or
+ *            NVFP4 code bytes [num_pages, Hkv, page_size, D/2]
+ * k/v_scales NVFP4 only: e4m3 block scales [num_pages, Hkv, page_size, D/16]
+ *            (NULL otherwise)
  * page_table int32 [B, max_pages]; kv_lens int32 [B]
  * sinks      float [Hq] attention-sink logits, or NULL for none
  * out        double [B, q_len, Hq, D]; lse double [B, q_len, Hq]
  */
 int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
-                             const void* v_pages, const int32_t* page_table,
+                             const void* v_pages, const void* k_scales,
+                             const void* v_scales, const int32_t* page_table,
                              const int32_t* kv_lens, int B, int q_len, int Hq,
                              int Hkv, int D, int page_size, int max_pages,
                              int num_pages, float scale, int causal_offset,
@@ -239,7 +282,8 @@ int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
   for (int b = 0; b < B; ++b)
     for (int i = 0; i < q_len; ++i)
       for (int h = 0; h < Hq; ++h) {
-        st = oracle_row(q, k_pages, v_pages, page_table, kv_lens, q_len, Hq, Hkv, D,
+        st = oracle_row(q, k_pages, v_pages, k_scales, v_scales, page_table, kv_lens,
+                        q_len, Hq, Hkv, D,
                         page_size, max_pages, num_pages, scale, causal_offset, window,
                         kv_dtype, kv_scale, tok_lo, tok_hi,
                         sinks ? (double)sinks[h] : -INFINITY, b, i, h, s, out, lse);
@@ -259,7 +303,8 @@ int oracle_paged_decode_attn(const uint16_t* q, const void* k_pages,
  * Without OpenMP support at build time it runs single-threaded.
  */
 int oracle_paged_decode_attn_mt(const uint16_t* q, const void* k_pages,
-                                const void* v_pages, const int32_t* page_table,
+                                const void* v_pages, const void* k_scales,
+                                const void* v_scales, const int32_t* page_table,
                                 const int32_t* kv_lens, int B, int q_len, int Hq,
                                 int Hkv, int D, int page_size, int max_pages,
                                 int num_pages, float scale, int causal_offset,
@@ -283,7 +328,8 @@ int oracle_paged_decode_attn_mt(const uint16_t* q, const void* k_pages,
       const int h = (int)(r % Hq);
       const int i = (int)((r / Hq) % q_len);
       const int b = (int)(r / ((int64_t)Hq * q_len));
-      local = oracle_row(q, k_pages, v_pages, page_table, kv_lens, q_len, Hq, Hkv, D,
+      local = oracle_row(q, k_pages, v_pages, k_scales, v_scales, page_table, kv_lens,
+                         q_len, Hq, Hkv, D,
                          page_size, max_pages, num_pages, scale, causal_offset, window,
                          kv_dtype, kv_scale, 0, -1, sinks ? (double)sinks[h] : -INFINITY,
                          b, i, h, s, out, lse);
@@ -332,6 +378,58 @@ uint8_t oracle_e4m3_encode(float x) {
 }
 
 /*
+ * E2M1 encoding of a float, from the format's definition: the code whose
+ * value is nearest to x, ties to the code with an even mantissa bit,
+ * magnitudes of 6 and above (and infinities) saturating to +-6; the sign
+ * bit follows x (so -0.0 and small negatives that round to zero give the
+ * negative zero code 0x8). NaN gives 0x7 (+6; the format has no NaN, and
+ * the library leaves NaN inputs unspecified). Walks all 8 non-negative codes.
+ */
+uint8_t oracle_e2m1_encode(float x) {
+  if (isnan(x)) return 0x7;
+  const int neg = signbit(x) ? 1 : 0;
+  const double a = fabs((double)x);
+  int best = 0;
+  if (a >= 6.0) {
+    best = 0x7;
+  } else {
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7; ++c) {
+      const double err = fabs(a - oracle_e2m1_to_double((uint8_t)c));
+      if (err < best_err || (err == best_err && (best & 1) == 1 && (c & 1) == 0)) {
+        best_err = err;
+        best = c;
+      }
+    }
+  }
+  return (uint8_t)(best | (neg << 3));
+}
+
+/*
+ * NVFP4 encoding of one block of 16 bf16 values (reading R23, the KV-cache
+ * producer's quantiser), every step in single precision:
+ *   q_d   = x_d / kv_scale                      (IEEE division)
+ *   amax  = max_d |q_d|
+ *   scale = e4m3(amax / 6)                      (nearest even, saturating)
+ *   code_d = e2m1(q_d / decode(scale))          (nearest even, saturating)
+ * A block whose scale decodes to zero stores every code as +0.
+ * codes[d] receives the 4-bit code of element d (one per byte here).
+ */
+void oracle_nvfp4_encode_block(const uint16_t* x, float kv_scale, uint8_t* codes,
+                               uint8_t* scale_code) {
+  float q[16];
+  float amax = 0.f;
+  for (int d = 0; d < 16; ++d) {
+    q[d] = (float)oracle_bf16_to_double(x[d]) / kv_scale;
+    const float a = fabsf(q[d]);
+    if (a > amax) amax = a;
+  }
+  *scale_code = oracle_e4m3_encode(amax / 6.0f);
+  const float sd = (float)oracle_e4m3_to_double(*scale_code);
+  for (int d = 0; d < 16; ++d) codes[d] = sd > 0.f ? oracle_e2m1_encode(q[d] / sd) : 0;
+}
+
+/*
  * Q as "native FP8 QK" uses it: each row of D bf16 values becomes
  * e4m3(q * 2^e) * 2^-e with 2^e the power of two that puts max|q| of the row
  * in [128, 256) (e = 7 - floor(log2 max|q|)); an all-zero row stays zero.
@@ -369,7 +467,11 @@ int oracle_quantize_q_e4m3(const uint16_t* q, int64_t rows, int D, uint16_t* q_o
  * single precision (the precision in which the quantised code is decided).
  *
  * k_new, v_new  bf16 bits [B, num_new, Hkv, D]
- * k/v_pages     bf16 bits or e4m3 bytes [num_pages, Hkv, P, D], updated in place
+ * k/v_pages     bf16 bits or e4m3 bytes [num_pages, Hkv, P, D], or NVFP4
+ *               code bytes [num_pages, Hkv, P, D/2], updated in place
+ * k/v_scales    NVFP4 only: e4m3 block scales [num_pages, Hkv, P, D/16],
+ *               updated in place (oracle_nvfp4_encode_block per 16 elements);
+ *               NULL otherwise
  * Returns ORACLE_BAD_PAGE (writing nothing more) at the first position past
  * the page table or page id out of range.
  */
@@ -377,11 +479,15 @@ int oracle_paged_kv_append(const uint16_t* k_new, const uint16_t* v_new,
                            const int32_t* page_table, const int32_t* kv_lens, int B,
                            int num_new, int Hkv, int D, int page_size, int max_pages,
                            int num_pages, int kv_dtype, float kv_scale, void* k_pages,
-                           void* v_pages) {
+                           void* v_pages, void* k_scales, void* v_scales) {
   if (B < 0 || num_new < 1 || Hkv < 1 || D < 1 || page_size < 1 || max_pages < 1 ||
       num_pages < 1)
     return ORACLE_BAD_ARG;
-  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3) return ORACLE_BAD_ARG;
+  if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8_E4M3 &&
+      kv_dtype != ORACLE_KV_NVFP4)
+    return ORACLE_BAD_ARG;
+  if (kv_dtype == ORACLE_KV_NVFP4 && (D % 16 != 0 || !k_scales || !v_scales))
+    return ORACLE_BAD_ARG;
   for (int b = 0; b < B; ++b) {
     for (int t = 0; t < num_new; ++t) {
       const int64_t pos = (int64_t)kv_lens[b] + t;
@@ -391,6 +497,20 @@ int oracle_paged_kv_append(const uint16_t* k_new, const uint16_t* v_new,
       for (int h = 0; h < Hkv; ++h) {
         const int64_t src = (((int64_t)b * num_new + t) * Hkv + h) * D;
         const int64_t dst = (((int64_t)page * Hkv + h) * page_size + pos % page_size) * D;
+        if (kv_dtype == ORACLE_KV_NVFP4) {
+          for (int blk = 0; blk < D / 16; ++blk) {
+            for (int which = 0; which < 2; ++which) {
+              const uint16_t* x = (which ? v_new : k_new) + src + 16 * blk;
+              uint8_t* codes = (uint8_t*)(which ? v_pages : k_pages);
+              uint8_t* scales = (uint8_t*)(which ? v_scales : k_scales);
+              uint8_t c[16];
+              oracle_nvfp4_encode_block(x, kv_scale, c, &scales[dst / 16 + blk]);
+              for (int d = 0; d < 16; d += 2)
+                codes[(dst + 16 * blk + d) / 2] = (uint8_t)(c[d] | (c[d + 1] << 4));
+            }
+          }
+          continue;
+        }
         for (int d = 0; d < D; ++d) {
           if (kv_dtype == ORACLE_KV_BF16) {
             ((uint16_t*)k_pages)[dst + d] = k_new[src + d];

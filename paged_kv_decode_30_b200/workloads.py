@@ -19,7 +19,15 @@ Two ways of filling the K/V pool:
 
 Pages that no sequence references, slots past ``kv_len`` in a sequence's last
 page, and (optionally) keys that no query row can see are filled with NaN
-(bf16 0x7FC0, e4m3 0x7F), so a kernel that reads or weights them shows it.
+(bf16 0x7FC0, e4m3 0x7F; NVFP4, whose codes have no NaN, gets NaN block
+scales), so a kernel that reads or weights them shows it.
+
+NVFP4 K/V (the cache builder's quantisation of the bf16 source, as the
+"b12x 0.30.0, Kernel inventory" FP4 rows and the "sglang profiler skill,
+fuse-overlap catalog" FP4 KV rows store it): packed E2M1 codes, two per
+byte with the even element in the low nibble, ``[num_pages, Hkv, P, D/2]``,
+plus one E4M3 scale per 16 consecutive elements of a row, ``[num_pages,
+Hkv, P, D/16]``, and the per-tensor ``kv_scale``.
 """
 
 from __future__ import annotations
@@ -32,12 +40,15 @@ import torch
 
 KV_BF16 = 0
 KV_FP8_E4M3 = 1
+KV_NVFP4 = 2
 CAUSAL_OFF = -1
 CAUSAL_BOTTOM_RIGHT = -2
 
 BF16_NAN_BITS = 0x7FC0
 E4M3_NAN_CODE = 0x7F
 E4M3_MAX = 448.0
+E2M1_MAX = 6.0
+NVFP4_BLOCK = 16
 
 
 @dataclasses.dataclass(frozen=True)
@@ -149,13 +160,17 @@ def generate(wl: Workload, device: str | torch.device = "cpu",
 
     Returns a dict with
       q           bf16 [B, q_len, Hq, D]
-      k_pages     bf16 or uint8 (e4m3 codes) [num_pages, Hkv, P, D]
+      k_pages     bf16 or uint8 (e4m3 codes) [num_pages, Hkv, P, D];
+                  NVFP4: uint8 packed E2M1 codes [num_pages, Hkv, P, D/2]
       v_pages     same
+      k_scales, v_scales  NVFP4: uint8 E4M3 block scales [num_pages, Hkv, P,
+                  D/16]; None otherwise
       page_table  int32 [B, max_pages] (unused slots -1)
       kv_lens     int32 [B]
       kv_scale    float (1.0 for bf16)
       k_dense / v_dense  (route "dense" only) lists of [Hkv, L_b, D] tensors
-                  holding the same values as the pages (bf16 or uint8)
+                  holding the same values as the pages (bf16 or uint8);
+                  NVFP4: lists of (codes [Hkv, L_b, D/2], scales [Hkv, L_b, D/16])
       workload    the Workload
     Generation happens on ``device`` with a generator seeded from the
     workload; the CPU and CUDA generators give different streams.
@@ -183,6 +198,7 @@ def generate(wl: Workload, device: str | torch.device = "cpu",
         off += n_pages[b]
 
     fp8 = wl.kv_dtype == KV_FP8_E4M3
+    nvfp4 = wl.kv_dtype == KV_NVFP4
     dense = (wl.route == "dense") if with_dense is None else with_dense
     shape = (num_pages, Hkv, P, D)
 
@@ -230,7 +246,20 @@ def generate(wl: Workload, device: str | torch.device = "cpu",
                     device=device, dtype=torch.float32).to(torch.bfloat16)
 
     kv_scale = 1.0
-    if fp8:
+    k_scales = v_scales = None
+    if nvfp4:
+        # per-tensor scale that puts the largest block scale at the top of
+        # the E4M3 range
+        amax = max(float(k_src.float().abs().max()) if k_src.numel() else 0.0,
+                   float(v_src.float().abs().max()) if v_src.numel() else 0.0)
+        kv_scale = float(torch.tensor(amax / (E2M1_MAX * E4M3_MAX), dtype=torch.float32)) or 1.0
+        k_pages, k_scales = encode_nvfp4(k_src, kv_scale)
+        v_pages, v_scales = encode_nvfp4(v_src, kv_scale)
+        if k_dense is not None:
+            k_dense = [encode_nvfp4(x, kv_scale) for x in k_dense]
+            v_dense = [encode_nvfp4(x, kv_scale) for x in v_dense]
+        del k_src, v_src
+    elif fp8:
         amax = max(float(k_src.float().abs().max()) if k_src.numel() else 0.0,
                    float(v_src.float().abs().max()) if v_src.numel() else 0.0)
         kv_scale = float(torch.tensor(amax / E4M3_MAX, dtype=torch.float32)) or 1.0
@@ -243,9 +272,12 @@ def generate(wl: Workload, device: str | torch.device = "cpu",
     else:
         k_pages, v_pages = k_src, v_src
 
-    _poison(wl, k_pages, v_pages, page_table, lens, n_pages, fp8)
+    if nvfp4:  # NaN lives in the block scales
+        _poison(wl, k_scales, v_scales, page_table, lens, n_pages, True)
+    else:
+        _poison(wl, k_pages, v_pages, page_table, lens, n_pages, fp8)
 
-    out = dict(q=q, k_pages=k_pages, v_pages=v_pages,
+    out = dict(q=q, k_pages=k_pages, v_pages=v_pages, k_scales=k_scales, v_scales=v_scales,
                page_table=page_table.to(device), kv_lens=lens.to(torch.int32).to(device),
                kv_scale=kv_scale, workload=wl, num_pages=num_pages,
                max_pages=max_pages)
@@ -259,6 +291,35 @@ def encode_e4m3(x: torch.Tensor, kv_scale: float) -> torch.Tensor:
     x / kv_scale, saturated to +-448, through torch's float8_e4m3fn cast."""
     y = (x.float() / kv_scale).clamp(-E4M3_MAX, E4M3_MAX)
     return y.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+# E2M1 magnitudes of codes 0..7 and the midpoints between neighbours.
+_E2M1_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+
+
+def encode_nvfp4(x: torch.Tensor, kv_scale: float):
+    """Quantise a bf16 source [..., D] to NVFP4: per block of 16 elements,
+    q = x / kv_scale, block scale = e4m3(max |q| / 6) through torch's
+    float8_e4m3fn cast, codes = the nearest E2M1 value of q / scale (ties to
+    the even code, saturating at 6; +0 codes where the scale is zero).
+    Returns (codes packed two per byte [..., D/2], scales [..., D/16])."""
+    D = x.shape[-1]
+    q = x.float() / kv_scale
+    blk = q.reshape(*q.shape[:-1], D // NVFP4_BLOCK, NVFP4_BLOCK)
+    amax = blk.abs().amax(dim=-1)
+    sc = (amax / E2M1_MAX).clamp(max=E4M3_MAX).to(torch.float8_e4m3fn)
+    sd = sc.float()[..., None]
+    y = torch.where(sd > 0, blk / torch.where(sd > 0, sd, torch.ones_like(sd)),
+                    torch.zeros_like(blk))
+    a = y.abs()
+    mids = torch.tensor(_E2M1_MIDPOINTS, dtype=torch.float32, device=x.device)
+    idx = torch.bucketize(a, mids)  # a <= mids[k] -> k
+    at = mids[idx.clamp(max=len(_E2M1_MIDPOINTS) - 1)]
+    idx = idx + ((a == at) & (idx % 2 == 1)).to(idx.dtype)  # ties to the even code
+    codes = (idx | torch.where(torch.signbit(y), 8, 0)).to(torch.uint8)
+    codes = codes.reshape(*q.shape[:-1], D)
+    packed = codes[..., 0::2] | (codes[..., 1::2] << 4)
+    return packed.contiguous(), sc.view(torch.uint8).contiguous()
 
 
 def _nan_fill(pages: torch.Tensor, fp8: bool, index):

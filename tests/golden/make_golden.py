@@ -1,7 +1,8 @@
 """Writes the hand-derived golden fixtures in this folder.
 
 Every expected value here is worked out by hand from a closed form or from the
-FP8 E4M3 format definition; the script only records those values as JSON.
+FP8 E4M3 / FP4 E2M1 format definitions; the script only records those values
+as JSON.
 It calls neither the CUDA library nor the oracle.
 
     python tests/golden/make_golden.py
@@ -111,6 +112,46 @@ def fixtures():
                   0xFE, 0x7F, 0xFF, 0x77, 0x30],
         "values": [0.0, -0.0, 0.001953125, 0.013671875, 0.015625, 1.0, 1.5, 2.0,
                    -2.0, 448.0, -448.0, "nan", "nan", 240.0, 0.5],
+    }
+    g["e2m1_codes"] = {
+        "source": "OCP FP4 E2M1: (-1)^s * 2^(e-1) * (1 + m/2) for exponent field e "
+                  "in 1..3; exponent 0 is subnormal m/2; no infinities or NaN; "
+                  "largest magnitude 6. Code bits s e1 e0 m. Values worked by hand.",
+        "codes": list(range(16)),
+        "values": [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,
+                   -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0],
+    }
+    g["nvfp4_blocks"] = {
+        "source": "NVFP4 block quantisation worked by hand: q = x / kv_scale; "
+                  "scale = e4m3(max|q| / 6) to nearest (ties even, saturating at "
+                  "448); code = e2m1(q / scale) to nearest, ties to the even "
+                  "mantissa bit, saturating at 6, sign kept; a zero scale stores "
+                  "+0 codes. Block 1: max|q| = 7, 7/6 = 1.1667 is nearest the "
+                  "e4m3 value 1.125 (code 0x39); q/1.125 gives 6.22 -> 6, 0.889 -> 1, "
+                  "2.5 -> 2 (tie, even), -0.222 -> -0, 0, -0, 0.5, 3.5 -> 4 (tie), "
+                  "-6.22 -> -6, 0.111 -> 0, 1.5, 4, -5 -> -4 (tie), 0.25 -> 0 (tie), "
+                  "2, -1.25 -> -1 (tie). Block 2: all zero, scale code 0, codes +0. "
+                  "Block 3: kv_scale 0.5, q = 6, -3, 1, 0 ... -> scale 1 (0x38). "
+                  "Block 4: kv_scale 2^-10, q = 2^22 -> scale saturates at 448 "
+                  "(0x7E), codes saturate at 6.",
+        "blocks": [
+            {"kv_scale": 1.0,
+             "x_bits": [bf(v) for v in (7.0, 1.0, 2.8125, -0.25, 0.0, -0.0, 0.5625,
+                                        3.9375, -7.0, 0.125, 1.6875, 4.5, -5.625,
+                                        0.28125, 2.25, -1.40625)],
+             "scale_code": 0x39,
+             "codes": [0x7, 0x2, 0x4, 0x8, 0x0, 0x8, 0x1, 0x6, 0xF, 0x0, 0x3, 0x6,
+                       0xE, 0x0, 0x4, 0xA]},
+            {"kv_scale": 1.0,
+             "x_bits": [bf(v) for v in (0.0, -0.0) * 8],
+             "scale_code": 0x00, "codes": [0x0] * 16},
+            {"kv_scale": 0.5,
+             "x_bits": [bf(v) for v in (3.0, -1.5, 0.5, 0.0) * 4],
+             "scale_code": 0x38, "codes": [0x7, 0xD, 0x2, 0x0] * 4},
+            {"kv_scale": 2.0 ** -10,
+             "x_bits": [bf(v) for v in (4096.0, -4096.0, 1.0, 0.0) * 4],
+             "scale_code": 0x7E, "codes": [0x7, 0xF, 0x4, 0x0] * 4},
+        ],
     }
     return g
 

@@ -27,6 +27,12 @@ What pins what:
   * append: new rows land where numpy indexing of the page table says
     (page_table[b][pos // P], slot pos % P), as torch-cast codes for FP8;
     every other slot is unchanged.
+  * NVFP4: E2M1 decode of all 16 codes and E2M1 encoding (nearest even,
+    saturating) against ml_dtypes' float4_e2m1fn (an independent
+    implementation) and hand-worked codes; the block quantiser against
+    hand-worked blocks and against a restatement built from numpy float32,
+    torch's float8_e4m3fn cast and ml_dtypes; brute force decodes NVFP4 K/V
+    through ml_dtypes and torch, never through the oracle.
 """
 
 from __future__ import annotations
@@ -35,6 +41,7 @@ import json
 import math
 import os
 
+import ml_dtypes
 import numpy as np
 import torch
 from scipy.special import logsumexp, softmax
@@ -78,7 +85,17 @@ SMALL_CASES = [
     W.Workload(name="peaked_d64_p32", batch=2, num_q_heads=4, num_kv_heads=1,
                head_dim=64, page_size=32, kv_lens=("fixed", [256, 130]),
                peaked_frac=0.05, route="dense", seed=18),
+    W.Workload(name="nvfp4_verify4_window64", batch=2, q_len=4, num_q_heads=8,
+               num_kv_heads=2, head_dim=32, page_size=16, kv_dtype=W.KV_NVFP4,
+               causal_offset=W.CAUSAL_BOTTOM_RIGHT, window=64,
+               kv_lens=("fixed", [100, 300]), route="dense", poison_invisible=True,
+               extra_pages=2, seed=19),
+    W.Workload(name="nvfp4_gqa4_d64_p8", batch=3, num_q_heads=8, num_kv_heads=2,
+               head_dim=64, page_size=8, kv_dtype=W.KV_NVFP4,
+               kv_lens=("fixed", [1, 37, 90]), route="dense", peaked_frac=0.05,
+               extra_pages=1, seed=20),
 ]
+NVFP4_CASES = [w for w in SMALL_CASES if w.kv_dtype == W.KV_NVFP4]
 
 
 def run_oracle(inp, lib, tok_range=None, **over):
@@ -87,17 +104,31 @@ def run_oracle(inp, lib, tok_range=None, **over):
               scale=W.scale_of(wl), causal_offset=wl.causal_offset,
               window=wl.window, kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"],
               tok_range=tok_range)
+    if inp.get("k_scales") is not None:
+        kw.update(k_scales=W.to_bits(inp["k_scales"]), v_scales=W.to_bits(inp["v_scales"]))
     kw.update(over)
     return orc.paged_decode_attn(
         W.to_bits(inp["q"]), W.to_bits(inp["k_pages"]), W.to_bits(inp["v_pages"]),
         inp["page_table"].cpu().numpy(), inp["kv_lens"].cpu().numpy(), lib=lib, **kw)
 
 
-def decode_dense(x: torch.Tensor, kv_dtype: int, kv_scale: float) -> np.ndarray:
-    """Values of a bf16 / e4m3-code tensor as float64, through torch's casts."""
+def e2m1_values(codes: np.ndarray) -> np.ndarray:
+    """float64 values of 4-bit E2M1 codes (one per byte), through ml_dtypes."""
+    return np.asarray(codes, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+
+
+def decode_dense(x, kv_dtype: int, kv_scale: float) -> np.ndarray:
+    """Values of a bf16 / e4m3-code / NVFP4 (codes, scales) tensor as float64,
+    through torch's and ml_dtypes' casts."""
     if kv_dtype == W.KV_BF16:
         return x.to(torch.float64).numpy()
-    return x.view(torch.float8_e4m3fn).to(torch.float64).numpy() * kv_scale
+    if kv_dtype == W.KV_FP8_E4M3:
+        return x.view(torch.float8_e4m3fn).to(torch.float64).numpy() * kv_scale
+    packed, scales = x
+    packed = packed.numpy()
+    codes = np.stack([packed & 0xF, packed >> 4], axis=-1).reshape(*packed.shape[:-1], -1)
+    blk = scales.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return e2m1_values(codes) * np.repeat(blk, 16, axis=-1) * kv_scale
 
 
 def visibility_matrix(L, q_len, causal_offset, window):
@@ -194,6 +225,76 @@ def check_decode_e4m3(lib):
             assert x == v and math.copysign(1, x) == math.copysign(1, v), (hex(c), x, v)
 
 
+def check_decode_e2m1(lib):
+    codes = np.arange(16, dtype=np.uint8)
+    ref = e2m1_values(codes)
+    got = np.array([orc.e2m1_to_double(int(c), lib=lib) for c in codes])
+    assert np.array_equal(got, ref), "e2m1 decode differs from ml_dtypes"
+    assert np.array_equal(np.signbit(got), np.signbit(ref))
+    g = load_golden("e2m1_codes")
+    for c, v in zip(g["codes"], g["values"]):
+        x = orc.e2m1_to_double(c, lib=lib)
+        assert x == v and math.copysign(1, x) == math.copysign(1, v), (hex(c), x, v)
+
+
+def check_e2m1_encode_vs_ml_dtypes(lib, n=50_000, seed=6):
+    """Against ml_dtypes' float4_e2m1fn cast (nearest even) of values clamped
+    to +-6 as the quantiser saturates: log-uniform magnitudes, every exact
+    midpoint between neighbouring codes, signed zeros and values past 6."""
+    g = torch.Generator().manual_seed(seed)
+    mag = torch.exp2(torch.rand(n, generator=g) * 8.0 - 4.0)          # 2^-4 .. 2^4
+    sign = torch.where(torch.rand(n, generator=g) < 0.5, -1.0, 1.0)
+    x = (mag * sign).float().numpy()
+    pos = e2m1_values(np.arange(8, dtype=np.uint8))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids, np.array([0.0, -0.0, 6.0, -6.0, 7.5, -1e30, 1e30],
+                                                 dtype=np.float32)]).astype(np.float32)
+    ref = np.clip(x, -6.0, 6.0).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    got = np.array([orc.e2m1_encode(float(v), lib=lib) for v in x], dtype=np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(x[i]), int(ref[i]), int(got[i])) for i in bad[:5]]
+
+
+def nvfp4_block_restated(x_bits: np.ndarray, kv_scale: float):
+    """The NVFP4 block rule restated with numpy float32 arithmetic, torch's
+    e4m3 cast and ml_dtypes' e2m1 cast."""
+    xf = torch.from_numpy(x_bits.astype(np.int32)).to(torch.int16).view(torch.bfloat16)
+    q = xf.float().numpy() / np.float32(kv_scale)
+    amax = np.float32(np.abs(q).max())
+    sc = torch.tensor([amax / np.float32(6.0)], dtype=torch.float32).clamp(max=448.0)
+    sc = sc.to(torch.float8_e4m3fn)
+    sd = np.float32(sc.float().item())
+    code = int(sc.view(torch.uint8).item())
+    if sd == 0:
+        return np.zeros(16, dtype=np.uint8), code
+    y = np.clip(q / sd, -6.0, 6.0).astype(np.float32)
+    return y.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF, code
+
+
+def check_nvfp4_block_golden(lib):
+    for blk in load_golden("nvfp4_blocks")["blocks"]:
+        codes, sc = orc.nvfp4_encode_block(np.array(blk["x_bits"], dtype=np.uint16),
+                                           blk["kv_scale"], lib=lib)
+        assert sc == blk["scale_code"], (hex(sc), hex(blk["scale_code"]))
+        assert codes.tolist() == blk["codes"], (codes.tolist(), blk["codes"])
+
+
+def check_nvfp4_block_vs_restated(lib, n=400, seed=9):
+    """Random blocks of mixed magnitude against the restated rule."""
+    g = torch.Generator().manual_seed(seed)
+    for k in range(n):
+        x = torch.randn(16, generator=g) * torch.exp2(torch.randint(-20, 20, (1,), generator=g).float())
+        if k % 7 == 0:
+            x[torch.rand(16, generator=g) < 0.3] = 0.0
+        bits = W.to_bits(x.to(torch.bfloat16))
+        kv_scale = float(torch.exp2(torch.randint(-12, 6, (1,), generator=g).float()) *
+                         (1 + torch.rand(1, generator=g)))
+        kv_scale = float(np.float32(kv_scale))
+        codes, sc = orc.nvfp4_encode_block(bits, kv_scale, lib=lib)
+        rc, rsc = nvfp4_block_restated(bits, kv_scale)
+        assert sc == rsc and np.array_equal(codes, rc), (k, kv_scale, sc, rsc, codes, rc)
+
+
 def check_bruteforce(wl, lib, tol=1e-12):
     inp = W.generate(wl)
     out, lse = run_oracle(inp, lib)
@@ -287,7 +388,8 @@ def check_poison_is_never_read(wl, lib):
     inp = W.generate(wl)
     out0, lse0 = run_oracle(inp, lib)
     clean = dict(inp)
-    for key in ("k_pages", "v_pages"):
+    keys = ("k_scales", "v_scales") if wl.kv_dtype == W.KV_NVFP4 else ("k_pages", "v_pages")
+    for key in keys:
         x = inp[key].clone()
         if wl.kv_dtype == W.KV_BF16:
             x[torch.isnan(x.float())] = 0
@@ -343,6 +445,14 @@ def run_all(lib):
     check_e4m3_encode_vs_torch(lib, n=20_000)
     check_append(lib, W.KV_BF16)
     check_append(lib, W.KV_FP8_E4M3)
+    check_decode_e2m1(lib)
+    check_e2m1_encode_vs_ml_dtypes(lib, n=5_000)
+    check_nvfp4_block_golden(lib)
+    check_nvfp4_block_vs_restated(lib, n=100)
+    check_append(lib, W.KV_NVFP4)
+    for wl in NVFP4_CASES:
+        check_bruteforce(wl, lib)
+        check_poison_is_never_read(wl, lib)
     for wl in (SMALL_CASES[2], SMALL_CASES[6], SMALL_CASES[7]):
         check_sink_bruteforce(wl, lib)
     check_quantize_q_vs_torch(lib)
@@ -381,37 +491,59 @@ def check_e4m3_encode_vs_torch(lib, n=200_000, seed=5):
 def check_append(lib, kv_dtype, seed=3):
     """New rows land at page_table[b][pos // P], slot pos % P for pos =
     kv_lens[b] + t (numpy indexing, independent of the oracle's loops), with
-    bf16 bits copied / e4m3 codes from torch's cast of the fp32 quotient;
-    every other slot is unchanged."""
+    bf16 bits copied / e4m3 codes from torch's cast of the fp32 quotient /
+    NVFP4 codes and block scales from the restated block rule; every other
+    slot is unchanged."""
     g = torch.Generator().manual_seed(seed)
-    B, T, Hkv, D, P, max_pages, num_pages = 3, 5, 2, 16, 8, 6, 30
+    B, T, Hkv, D, P, max_pages, num_pages = 3, 5, 2, 32, 8, 6, 30
     kv_lens = np.array([0, 7, 22], dtype=np.int32)
     page_table = torch.randperm(num_pages, generator=g)[:B * max_pages].reshape(B, max_pages)
     page_table = page_table.to(torch.int32).numpy()
     k_new = torch.randn((B, T, Hkv, D), generator=g).to(torch.bfloat16)
     v_new = torch.randn((B, T, Hkv, D), generator=g).to(torch.bfloat16)
     fp8 = kv_dtype == W.KV_FP8_E4M3
-    dt = np.uint8 if fp8 else np.uint16
-    k_pages = np.random.default_rng(seed).integers(0, 255, (num_pages, Hkv, P, D)).astype(dt)
-    v_pages = np.random.default_rng(seed + 1).integers(0, 255, (num_pages, Hkv, P, D)).astype(dt)
+    nv = kv_dtype == W.KV_NVFP4
+    dt = np.uint16 if kv_dtype == W.KV_BF16 else np.uint8
+    Dp = D // 2 if nv else D
+    k_pages = np.random.default_rng(seed).integers(0, 255, (num_pages, Hkv, P, Dp)).astype(dt)
+    v_pages = np.random.default_rng(seed + 1).integers(0, 255, (num_pages, Hkv, P, Dp)).astype(dt)
     scale = 0.0123
-    kp, vp = orc.paged_kv_append(W.to_bits(k_new), W.to_bits(v_new), page_table, kv_lens,
-                                 k_pages, v_pages, page_size=P, kv_dtype=kv_dtype,
-                                 kv_scale=scale, lib=lib)
+    extra = {}
+    if nv:
+        extra = dict(
+            k_scales=np.random.default_rng(seed + 2).integers(0, 255, (num_pages, Hkv, P, D // 16)).astype(np.uint8),
+            v_scales=np.random.default_rng(seed + 3).integers(0, 255, (num_pages, Hkv, P, D // 16)).astype(np.uint8))
+    res = orc.paged_kv_append(W.to_bits(k_new), W.to_bits(v_new), page_table, kv_lens,
+                              k_pages, v_pages, page_size=P, kv_dtype=kv_dtype,
+                              kv_scale=scale, lib=lib, **extra)
 
     def coded(x):
+        if nv:  # [T, Hkv, D] -> packed codes [T, Hkv, D/2], scales [T, Hkv, D/16]
+            bits = W.to_bits(x).reshape(-1, 16)
+            out = [nvfp4_block_restated(b_, scale) for b_ in bits]
+            c = np.stack([o[0] for o in out]).reshape(*x.shape)
+            sc = np.array([o[1] for o in out], dtype=np.uint8).reshape(*x.shape[:-1], D // 16)
+            return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8), sc
         if not fp8:
             return W.to_bits(x)
         y = (x.float() / scale).clamp(-448.0, 448.0)
         return y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
     ek, ev = k_pages.copy(), v_pages.copy()
+    if nv:
+        eks, evs = extra["k_scales"].copy(), extra["v_scales"].copy()
     for b in range(B):
         pos = kv_lens[b] + np.arange(T)
         pages = page_table[b, pos // P]
-        ek[pages, :, pos % P, :] = coded(k_new[b])
-        ev[pages, :, pos % P, :] = coded(v_new[b])
-    assert np.array_equal(kp, ek) and np.array_equal(vp, ev)
+        if nv:
+            ek[pages, :, pos % P, :], eks[pages, :, pos % P, :] = coded(k_new[b])
+            ev[pages, :, pos % P, :], evs[pages, :, pos % P, :] = coded(v_new[b])
+        else:
+            ek[pages, :, pos % P, :] = coded(k_new[b])
+            ev[pages, :, pos % P, :] = coded(v_new[b])
+    assert np.array_equal(res[0], ek) and np.array_equal(res[1], ev)
+    if nv:
+        assert np.array_equal(res[2], eks) and np.array_equal(res[3], evs)
 
 
 # ---------------------------------------------------------------------------

@@ -138,6 +138,20 @@ MUTATIONS = {
     "sink_empty_row": ("*lrow = sink;", "*lrow = -INFINITY;"),
     "quantize_q_scale_off_by_one": ("const int e = mx > 0.0 ? 7 - ilogb(mx) : 0;",
                                     "const int e = mx > 0.0 ? 8 - ilogb(mx) : 0;"),
+    "e2m1_bias": ("mag = ldexp(1.0 + (double)m / 2.0, e - 1);",
+                  "mag = ldexp(1.0 + (double)m / 2.0, e - 2);"),
+    "nvfp4_nibble_order": ("(index % 2) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF)",
+                           "(index % 2) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4)"),
+    "nvfp4_block_index": ("((const uint8_t*)scales)[index / 16]",
+                          "((const uint8_t*)scales)[index / 32]"),
+    "nvfp4_block_scale_dropped": ("return oracle_e2m1_to_double(code) * block * kv_scale;",
+                                  "return oracle_e2m1_to_double(code) * kv_scale;"),
+    "e2m1_ties_to_odd": ("(best & 1) == 1 && (c & 1) == 0", "(best & 1) == 0 && (c & 1) == 1"),
+    "nvfp4_amax_over_4": ("oracle_e4m3_encode(amax / 6.0f)", "oracle_e4m3_encode(amax / 4.0f)"),
+    "nvfp4_zero_scale_keeps_sign": ("sd > 0.f ? oracle_e2m1_encode(q[d] / sd) : 0;",
+                                    "sd > 0.f ? oracle_e2m1_encode(q[d] / sd) : (signbit(q[d]) ? 8 : 0);"),
+    "nvfp4_append_nibbles_swapped": ("(uint8_t)(c[d] | (c[d + 1] << 4))",
+                                     "(uint8_t)(c[d + 1] | (c[d] << 4))"),
 }
 
 
@@ -177,9 +191,37 @@ def test_e4m3_encode_matches_torch_cast(lib):
     pins.check_e4m3_encode_vs_torch(lib)
 
 
-@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3])
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3, W.KV_NVFP4])
 def test_append_places_rows_by_page_table(lib, kv_dtype):
     pins.check_append(lib, kv_dtype)
+
+
+def test_e2m1_decode_matches_ml_dtypes_and_format(lib):
+    pins.check_decode_e2m1(lib)
+
+
+def test_e2m1_encode_matches_ml_dtypes_cast(lib):
+    pins.check_e2m1_encode_vs_ml_dtypes(lib)
+
+
+def test_nvfp4_block_quantiser_hand_worked(lib):
+    pins.check_nvfp4_block_golden(lib)
+
+
+def test_nvfp4_block_quantiser_matches_restatement(lib):
+    pins.check_nvfp4_block_vs_restated(lib)
+
+
+@pytest.mark.parametrize("wl", pins.NVFP4_CASES, ids=lambda w: w.name)
+def test_nvfp4_poisoned_scales_are_never_read(lib, wl):
+    pins.check_poison_is_never_read(wl, lib)
+
+
+def test_nvfp4_multithreaded_oracle_is_bit_identical(lib):
+    inp = W.generate(pins.NVFP4_CASES[0], device="cpu")
+    ref = pins.run_oracle(inp, lib)
+    got = pins.run_oracle(inp, lib, threads=4)
+    assert np.array_equal(ref[0], got[0]) and np.array_equal(ref[1], got[1])
 
 
 @pytest.mark.parametrize("wl", [pins.SMALL_CASES[i] for i in (0, 2, 3, 6, 7, 8)], ids=lambda w: w.name)
