@@ -1,6 +1,8 @@
-// paged_decode_attn_no_alloc: the paged decode call with its split-KV
-// partials kept in a fixed device array that ships with the library, for
-// callers that cannot allocate device memory.
+// paged_decode_attn_no_alloc: the paged decode call with its whole workspace
+// (the tensor-core kernel's counter header, work-queue order and FP8 Q
+// operand images, and the split-KV partials) kept in a fixed device array
+// that ships with the library, for callers that cannot allocate device
+// memory. The limit applies to paged_decode_attn_workspace_bytes(params).
 //
 // Who cannot allocate: a serving engine that reserves nearly all of HBM for
 // its own KV-cache pool at start-up and lets no library allocate afterwards;
