@@ -4,7 +4,10 @@ One step = one call of ``paged_decode_attn`` (split kernel, plus the merge
 kernel when the planner splits) over one batch of synthetic inputs that are
 already resident in HBM. Default workload: B=128 sequences, 32 query / 8 KV
 heads, head_dim 128, page_size 16, kv_len 8192, bf16 K/V (4.3 GB of K/V, far
-larger than L2, so no flush is needed between steps).
+larger than L2, so no flush is needed between steps). After it, every other
+workload is timed in the same process at the same --steps / --warmup, each
+with its own L2 policy (pools under 1 GiB rotate among copies; tiny ones get
+an L2 flush before every step), into the line's ``workloads`` object.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed
@@ -60,6 +63,10 @@ def parse_args(argv=None):
                     help="FP8 K/V: q enters QK^T as one e4m3 term (changes the result)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the read-only HBM probe and the CUDA-graph replay (profiling runs)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only --workload (not every workload)")
+    ap.add_argument("--cpu-seconds-per-workload", type=float, default=3.0,
+                    help="bound of each workload entry's CPU oracle sample")
     return ap.parse_args(argv)
 
 
@@ -218,6 +225,10 @@ def oracle_units(inp, units):
         idx = pt[b, :n].to(torch.int64).to(inp["k_pages"].device)
         kp = inp["k_pages"][idx, g: g + 1].contiguous()
         vp = inp["v_pages"][idx, g: g + 1].contiguous()
+        sc = {}
+        if inp.get("k_scales") is not None:
+            sc = dict(k_scales=W.to_bits(inp["k_scales"][idx, g: g + 1].contiguous()),
+                      v_scales=W.to_bits(inp["v_scales"][idx, g: g + 1].contiguous()))
         q = inp["q"][b: b + 1, :, g * G: (g + 1) * G].contiguous()
         args = (W.to_bits(q), W.to_bits(kp), W.to_bits(vp),
                 torch.arange(n, dtype=torch.int32).reshape(1, n).numpy(),
@@ -225,7 +236,7 @@ def oracle_units(inp, units):
         t0 = time.perf_counter()
         orc.paged_decode_attn(*args, num_kv_heads=1, page_size=P, scale=W.scale_of(wl),
                               causal_offset=wl.causal_offset, window=wl.window,
-                              kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"])
+                              kv_dtype=wl.kv_dtype, kv_scale=inp["kv_scale"], **sc)
         elapsed += time.perf_counter() - t0
     return elapsed
 
@@ -239,11 +250,14 @@ def oracle_sequences_mt(inp, first: int, count: int, threads: int) -> float:
     args = (W.to_bits(inp["q"][sl].contiguous()), W.to_bits(inp["k_pages"]),
             W.to_bits(inp["v_pages"]), inp["page_table"][sl].contiguous().cpu().numpy(),
             inp["kv_lens"][sl].contiguous().cpu().numpy())
+    sc = {}
+    if inp.get("k_scales") is not None:
+        sc = dict(k_scales=W.to_bits(inp["k_scales"]), v_scales=W.to_bits(inp["v_scales"]))
     t0 = time.perf_counter()
     orc.paged_decode_attn(*args, num_kv_heads=wl.num_kv_heads, page_size=wl.page_size,
                           scale=W.scale_of(wl), causal_offset=wl.causal_offset,
                           window=wl.window, kv_dtype=wl.kv_dtype,
-                          kv_scale=inp["kv_scale"], threads=threads)
+                          kv_scale=inp["kv_scale"], threads=threads, **sc)
     return time.perf_counter() - t0
 
 
@@ -252,6 +266,30 @@ def host_threads() -> int:
         return len(os.sched_getaffinity(0))
     except AttributeError:
         return os.cpu_count() or 1
+
+
+def cpu_baseline_mt(inp, seconds: float):
+    """The oracle on every host core (OpenMP, one output row per task) on
+    whole sequences of the workload, for about `seconds`."""
+    wl = inp["workload"]
+    threads = host_threads()
+    seqs, mt_elapsed = 0, 0.0
+    # the K/V pools go to the host once; each call then takes whole sequences
+    host = dict(inp, q=inp["q"].cpu(), k_pages=inp["k_pages"].cpu(),
+                v_pages=inp["v_pages"].cpu(), page_table=inp["page_table"].cpu(),
+                kv_lens=inp["kv_lens"].cpu())
+    if inp.get("k_scales") is not None:
+        host.update(k_scales=inp["k_scales"].cpu(), v_scales=inp["v_scales"].cpu())
+    while mt_elapsed < seconds and seqs < wl.batch:
+        n = min(max(1, threads // max(1, wl.num_q_heads * wl.q_len) + 1), wl.batch - seqs)
+        mt_elapsed += oracle_sequences_mt(host, seqs, n, threads)
+        seqs += n
+    return {
+        "value": seqs * wl.q_len / mt_elapsed, "unit": "tokens/s", "cores": threads,
+        "kind": "oracle",
+        "sample": (f"{seqs} full sequences (all heads) of {wl.name}, fp64 C oracle on "
+                   f"{threads} OpenMP threads (one output row per task), {mt_elapsed:.2f} s"),
+    }
 
 
 def cpu_baseline(inp, seconds: float):
@@ -271,23 +309,9 @@ def cpu_baseline(inp, seconds: float):
                    f"({units / wl.num_kv_heads:.3f} full sequences, all heads), "
                    f"single-threaded fp64 C oracle, {elapsed:.1f} s"),
     }
-    threads = host_threads()
-    seqs, mt_elapsed = 0, 0.0
-    # the K/V pools go to the host once; each call then takes whole sequences
-    host = dict(inp, q=inp["q"].cpu(), k_pages=inp["k_pages"].cpu(),
-                v_pages=inp["v_pages"].cpu(), page_table=inp["page_table"].cpu(),
-                kv_lens=inp["kv_lens"].cpu())
-    while mt_elapsed < seconds and seqs < wl.batch:
-        n = min(max(1, threads // max(1, wl.num_q_heads * wl.q_len) + 1), wl.batch - seqs)
-        mt_elapsed += oracle_sequences_mt(host, seqs, n, threads)
-        seqs += n
-    return {
-        "value": seqs * wl.q_len / mt_elapsed, "unit": "tokens/s", "cores": threads,
-        "kind": "oracle",
-        "sample": (f"{seqs} full sequences (all heads) of {wl.name}, fp64 C oracle on "
-                   f"{threads} OpenMP threads (one output row per task), {mt_elapsed:.1f} s"),
-        "single_thread": single,
-    }
+    mt = cpu_baseline_mt(inp, seconds)
+    mt["single_thread"] = single
+    return mt
 
 
 # ---------------------------------------------------------------------------
@@ -326,74 +350,102 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, rank, world, local):
-    if not torch.cuda.is_available():
-        raise RuntimeError("bench.py needs a CUDA device (the library has no CPU path)")
-    B.load()
-    wl = W.ALL[args.workload]
-    if args.batch:
-        wl = wl.with_(batch=args.batch, name=f"{wl.name}_batch{args.batch}")
-    dev = torch.device("cuda", torch.cuda.current_device())
-    inp = W.generate(wl, device=dev, seed=wl.seed + rank)
-    scale = W.scale_of(wl)
-    q, kp, vp = inp["q"], inp["k_pages"], inp["v_pages"]
-    pt, kl = inp["page_table"], inp["kv_lens"]
-    max_len = int(kl.max().item())
-    out = torch.empty((wl.batch, wl.q_len, wl.num_q_heads, wl.head_dim), dtype=torch.float32, device=dev)
-    lse = torch.empty((wl.batch, wl.q_len, wl.num_q_heads), dtype=torch.float32, device=dev)
+L2_FLUSH_BYTES = 256 * 1024 * 1024
+# K/V pools under this size are timed rotating among copies of themselves,
+# so consecutive steps never find their K/V in L2.
+ROTATE_BELOW_BYTES = 1 << 30
+ROTATE_MIN_POOL_BYTES = 16 * 1024 * 1024  # smaller pools: flush L2 instead
+
+
+def run_flags(args) -> int:
     flags = {"auto": 0, "tensor_cores": B.PDA_FLAG_TENSOR_CORES,
              "cuda_cores": B.PDA_FLAG_CUDA_CORES}[args.kernel]
     if args.fused_merge:
         flags |= B.PDA_FLAG_FUSED_MERGE
     if args.native_fp8_qk:
         flags |= B.PDA_FLAG_NATIVE_FP8_QK
+    return flags
+
+
+def prepare(wl, dev, rank, splits, flags):
+    """Inputs of one workload resident in HBM, the call's arguments, and the
+    L2 policy of its timed region: pools of 1 GiB or more are read as they
+    are; smaller pools (down to 16 MiB) rotate among enough copies that a
+    copy comes back only after 1 GiB of other K/V; tiny pools get a 256 MiB
+    write before every timed step instead (outside the step's events)."""
+    inp = W.generate(wl, device=dev, seed=wl.seed + rank)
+    scale = W.scale_of(wl)
+    kp, vp, pt, kl = inp["k_pages"], inp["v_pages"], inp["page_table"], inp["kv_lens"]
+    max_len = int(kl.max().item())
+    out = torch.empty((wl.batch, wl.q_len, wl.num_q_heads, wl.head_dim), dtype=torch.float32,
+                      device=dev)
+    lse = torch.empty((wl.batch, wl.q_len, wl.num_q_heads), dtype=torch.float32, device=dev)
     kw = dict(num_kv_heads=wl.num_kv_heads, scale=scale, causal_offset=wl.causal_offset,
               window=wl.window, kv_scale=inp["kv_scale"], max_kv_len=max_len,
-              num_splits=args.splits, flags=flags)
+              num_splits=splits, flags=flags)
     params = B.make_params(
         batch=wl.batch, q_len=wl.q_len, num_q_heads=wl.num_q_heads,
         num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim, page_size=wl.page_size,
         max_pages_per_seq=pt.shape[1], num_pages=kp.shape[0], scale=scale,
         causal_offset=wl.causal_offset, window=wl.window, kv_dtype=wl.kv_dtype,
-        kv_scale=inp["kv_scale"], max_kv_len=max_len, num_splits=args.splits, flags=flags)
+        kv_scale=inp["kv_scale"], max_kv_len=max_len, num_splits=splits, flags=flags)
     kernel_name = B.KERNEL_NAMES.get(B.plan_kernel(params), "unknown")
-    ws_bytes = B.workspace_bytes(params)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        return B.paged_decode_attn(q, kp, vp, pt, kl, out=out, lse=lse, workspace=ws, **kw)[2]
-
-    # K/V smaller than twice the L2 (126 MB) could stay cached between
-    # steps: then every timed step is preceded by a 256 MiB write (outside
-    # the step's events) and the value comes from the per-step events.
-    _, kv_bytes0 = algorithmic_bytes(wl, kl.tolist())
+    ws = torch.empty(max(B.workspace_bytes(params), 1), dtype=torch.uint8, device=dev)
+    pool_bytes = kp.numel() * kp.element_size() * 2
+    pools = [(kp, vp)]
     flush = None
-    if kv_bytes0 < 2 * L2_BYTES:
-        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    if pool_bytes >= ROTATE_BELOW_BYTES:
+        l2 = (f"no flush: the K/V pools ({pool_bytes / 1e9:.2f} GB) are more than 8x the "
+              "L2 (126 MB)")
+    elif pool_bytes >= ROTATE_MIN_POOL_BYTES:
+        n = max(2, -(-ROTATE_BELOW_BYTES // pool_bytes))
+        pools += [(kp.clone(), vp.clone()) for _ in range(n - 1)]
+        l2 = (f"rotating {n} copies of the K/V pools ({pool_bytes / 1e9:.3f} GB each): "
+              f"step i reads copy i mod {n}, so a copy returns after "
+              f"{(n - 1) * pool_bytes / 1e9:.2f} GB of other K/V")
+    else:
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        l2 = ("flushed before every timed step (256 MiB write, outside the step's events; "
+              "the time is the sum of the per-step events)")
+    return dict(wl=wl, inp=inp, out=out, lse=lse, kw=kw, ws=ws, pools=pools, flush=flush,
+                l2=l2, kernel_name=kernel_name, max_len=max_len)
 
-    splits = step()
+
+def call(ctx, i=0):
+    kp, vp = ctx["pools"][i % len(ctx["pools"])]
+    inp = ctx["inp"]
+    return B.paged_decode_attn(inp["q"], kp, vp, inp["page_table"], inp["kv_lens"],
+                               out=ctx["out"], lse=ctx["lse"], workspace=ctx["ws"],
+                               **ctx["kw"])[2]
+
+
+def time_steps(ctx, steps, warmup, world, local):
+    """W warm-up steps, then exactly `steps` steps between a barrier and a
+    synchronize on both sides, each step bracketed by CUDA events on the
+    launching stream. Returns (elapsed ms, per-step ms, clocks, splits)."""
+    stream = torch.cuda.current_stream()
+    splits = call(ctx)
     torch.cuda.synchronize()
     if B.last_device_error() != 0:
-        raise RuntimeError("device error word set after the first call")
-    for _ in range(max(args.warmup, 3)):
-        step()
-
+        raise RuntimeError(f"{ctx['wl'].name}: device error word set after the first call")
+    for i in range(max(warmup, 3)):
+        call(ctx, i + 1)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)  # let the sampler start before the timed region
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    flush = ctx["flush"]
     t_begin.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         if flush is not None:
             flush.fill_(i & 0xFF)
         starts[i].record(stream)
-        step()
+        call(ctx, i)
         ends[i].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -404,19 +456,104 @@ def run_ours(args, rank, world, local):
     if flush is not None:  # the flushes are not part of the job
         elapsed_ms = sum(step_ms)
     if B.last_device_error() != 0:
-        raise RuntimeError("device error word set during the timed region")
+        raise RuntimeError(f"{ctx['wl'].name}: device error word set during the timed region")
+    return max_over_ranks(elapsed_ms, world), step_ms, clocks, splits
 
-    elapsed_ms = max_over_ranks(elapsed_ms, world)
+
+def launches_per_step(kernel_name, splits, fused_merge):
+    """Our kernels per call: the tensor-core kernel runs after its prologue
+    kernel (counters, queue order, FP8 Q images); the merge kernel follows
+    when the splits are merged apart."""
+    merge = splits > 1 and not (kernel_name == "split_tma_kernel" and fused_merge)
+    return (2 if kernel_name == "split_tma_kernel" else 1) + (1 if merge else 0), merge
+
+
+def graph_replay(ctx, steps, world):
+    """One call captured in a CUDA graph and replayed (no host launch gaps;
+    L2 not flushed between replays)."""
+    stream = torch.cuda.current_stream()
+    wl = ctx["wl"]
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(ctx)
+        for _ in range(3):
+            g.replay()
+        n_g = max(20, min(steps, 500))
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(n_g):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        g_ms = g0.elapsed_time(g1) / n_g
+        del g
+        return {"ms_per_step": g_ms, "value": wl.batch * wl.q_len * world / (g_ms / 1e3),
+                "unit": "tokens/s", "replays": n_g, "l2": "warm (no flush between replays)"}
+    except RuntimeError as e:
+        return {"error": str(e).splitlines()[0][:200]}
+
+
+def workload_entry(ctx, args, world, local, peak, probe_gbs, fused_merge, with_cpu):
+    """Time one workload; its numbers as one entry of the line's
+    `workloads` object."""
+    wl = ctx["wl"]
+    elapsed_ms, step_ms, clocks, splits = time_steps(ctx, args.steps, args.warmup, world, local)
+    alg_bytes, kv_bytes = algorithmic_bytes(wl, ctx["inp"]["kv_lens"].tolist())
+    avg_ms = statistics.mean(step_ms)
+    gbs = alg_bytes / (avg_ms / 1e3) / 1e9
+    per_step, merge = launches_per_step(ctx["kernel_name"], splits, fused_merge)
+    entry = {
+        "ms_per_step": elapsed_ms / args.steps,
+        "tokens_per_s": wl.batch * wl.q_len * args.steps * world / (elapsed_ms / 1e3),
+        "algorithmic_bytes_per_step": alg_bytes,
+        "avg_launch_ms": avg_ms,
+        "gb_s": gbs,
+        "frac_of_copy": gbs / peak,
+        "frac_of_8tbs_spec": gbs / 8000.0,
+        "frac_of_read_probe": gbs / probe_gbs if probe_gbs else None,
+        "kernel": ctx["kernel_name"] + (" + merge_states_kernel" if merge else ""),
+        "splits": splits,
+        "gpu_launches": per_step * args.steps,
+        "steps": args.steps, "warmup": args.warmup,
+        "batch": wl.batch, "q_len": wl.q_len, "num_q_heads": wl.num_q_heads,
+        "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "page_size": wl.page_size,
+        "kv_dtype": {W.KV_BF16: "bf16", W.KV_FP8_E4M3: "fp8_e4m3"}.get(wl.kv_dtype, wl.kv_dtype),
+        "l2": ctx["l2"],
+        "clocks": clocks,
+        "graph": None if args.no_extras else graph_replay(ctx, args.steps, world),
+        "traffic": recorded_traffic(wl.name, ctx["kernel_name"]),
+    }
+    if with_cpu:
+        entry["cpu_baseline"] = cpu_baseline_mt(ctx["inp"], args.cpu_seconds_per_workload)
+    return entry
+
+
+def run_ours(args, rank, world, local):
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device (the library has no CPU path)")
+    B.load()
+    wl = W.ALL[args.workload]
+    if args.batch:
+        wl = wl.with_(batch=args.batch, name=f"{wl.name}_batch{args.batch}")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flags = run_flags(args)
+    ctx = prepare(wl, dev, rank, args.splits, flags)
+    inp, out, lse, ws, kw = ctx["inp"], ctx["out"], ctx["lse"], ctx["ws"], ctx["kw"]
+    q, kp, vp = inp["q"], inp["k_pages"], inp["v_pages"]
+    pt, kl = inp["page_table"], inp["kv_lens"]
+    max_len = ctx["max_len"]
+    kernel_name = ctx["kernel_name"]
+    stream = torch.cuda.current_stream()
+
+    elapsed_ms, step_ms, clocks, splits = time_steps(ctx, args.steps, args.warmup, world, local)
     tokens_per_step = wl.batch * wl.q_len
     value = tokens_per_step * args.steps * world / (elapsed_ms / 1e3)
     alg_bytes, kv_bytes = algorithmic_bytes(wl, kl.tolist())
     avg_launch_ms = statistics.mean(step_ms)
     achieved = alg_bytes / (avg_launch_ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
-    merge_launched = splits > 1 and not (kernel_name == "split_tma_kernel" and args.fused_merge)
-    # the tensor-core kernel runs after its prologue kernel (counters, queue
-    # order, FP8 Q images); the merge kernel follows when splits are merged apart
-    launches_per_step = (2 if kernel_name == "split_tma_kernel" else 1) + (1 if merge_launched else 0)
+    per_step, merge_launched = launches_per_step(kernel_name, splits, args.fused_merge)
 
     # Read-only HBM probe in the same run (our streaming-load kernel over a
     # 4 GiB buffer, larger than L2): the ceiling for a kernel that only reads.
@@ -440,30 +577,7 @@ def run_ours(args, rank, world, local):
     except (RuntimeError, B.PdaError) as e:  # out of memory: report none
         print(f"read probe skipped: {e}", file=sys.stderr)
 
-    # One call captured in a CUDA graph and replayed (no host launch gaps;
-    # L2 not flushed between replays).
-    graph = None
-    try:
-        if args.no_extras:
-            raise RuntimeError("skipped (--no-extras)")
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step()
-        for _ in range(3):
-            g.replay()
-        n_g = max(20, min(args.steps, 500))
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        g0.record(stream)
-        for _ in range(n_g):
-            g.replay()
-        g1.record(stream)
-        torch.cuda.synchronize()
-        g_ms = g0.elapsed_time(g1) / n_g
-        graph = {"ms_per_step": g_ms, "value": tokens_per_step * world / (g_ms / 1e3),
-                 "unit": "tokens/s", "replays": n_g, "l2": "warm (no flush between replays)"}
-        del g
-    except RuntimeError as e:
-        graph = {"error": str(e).splitlines()[0][:200]}
+    graph = None if args.no_extras else graph_replay(ctx, args.steps, world)
 
     # End to end through the public API with host buffers: every step copies
     # the step's inputs (q, page table, kv lengths) from pinned host memory
@@ -544,6 +658,43 @@ def run_ours(args, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, args.cpu_seconds)
 
+    # Every workload, each timed in this process at the same --steps and
+    # --warmup with its own L2 policy (the line's top level is the one
+    # above; its entry repeats those numbers).
+    workloads = None
+    if not (args.no_workloads or args.batch):
+        workloads = {}
+        with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+        for name, other in W.ALL.items():
+            if name == wl.name:
+                entry = {
+                    "ms_per_step": elapsed_ms / args.steps, "tokens_per_s": value,
+                    "algorithmic_bytes_per_step": alg_bytes, "avg_launch_ms": avg_launch_ms,
+                    "gb_s": achieved, "frac_of_copy": achieved / peak,
+                    "frac_of_8tbs_spec": achieved / 8000.0,
+                    "frac_of_read_probe": achieved / probe_gbs if probe_gbs else None,
+                    "kernel": kernel_name + (" + merge_states_kernel" if merge_launched else ""),
+                    "splits": splits, "gpu_launches": per_step * args.steps,
+                    "steps": args.steps, "warmup": args.warmup, "batch": wl.batch,
+                    "q_len": wl.q_len, "num_q_heads": wl.num_q_heads,
+                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                    "page_size": wl.page_size,
+                    "kv_dtype": {W.KV_BF16: "bf16", W.KV_FP8_E4M3: "fp8_e4m3"}.get(
+                        wl.kv_dtype, wl.kv_dtype),
+                    "l2": ctx["l2"], "clocks": clocks, "graph": graph,
+                    "traffic": recorded_traffic(wl.name, kernel_name),
+                    "cpu_baseline": (cpu_baseline_mt(inp, args.cpu_seconds_per_workload)
+                                     if with_cpu else None),
+                    "top_level": True,
+                }
+            else:
+                octx = prepare(other, dev, rank, args.splits, flags)
+                entry = workload_entry(octx, args, world, local, peak, probe_gbs,
+                                       args.fused_merge, with_cpu)
+                del octx
+                torch.cuda.empty_cache()
+            workloads[name] = entry
+
     if rank != 0:
         return
     line = {
@@ -566,10 +717,7 @@ def run_ours(args, rank, world, local):
             "kv_len": max_len if wl.kv_lens[0] == "const" else str(wl.kv_lens),
             "causal_offset": wl.causal_offset, "window": wl.window,
             "num_splits": splits, "parallelism": f"replicas x{world}",
-            "l2": ("flushed before every timed step (256 MiB write, outside the step's "
-                   "events; value from the per-step events)") if flush is not None
-                  else f"no flush: K/V read per step ({kv_bytes / 1e9:.2f} GB) is more than "
-                       "twice the L2",
+            "l2": ctx["l2"],
             "algorithmic_bytes_per_step": alg_bytes,
         },
         "roofline": {
@@ -584,12 +732,13 @@ def run_ours(args, rank, world, local):
             "frac_of_read_probe": achieved / probe_gbs if probe_gbs else None,
             "avg_launch_ms": avg_launch_ms,
         },
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": per_step * args.steps,
         "clocks": clocks,
         "graph": graph,
         "kv_append": kv_append,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "workloads": workloads,
     }
     print(json.dumps(line), flush=True)
 

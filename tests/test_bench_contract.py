@@ -47,3 +47,28 @@ def test_bench_line_carries_the_contract_fields():
     assert d["gpu_launches"] >= d["steps"]
     ck = d["clocks"]
     assert ck["sm_max_mhz"] > 0 and isinstance(ck["reasons"], list)
+    # every workload, timed in the same run, each with its L2 policy
+    wls = d["workloads"]
+    assert set(wls) == {"tiny_b2_gqa4_d64_p16", "varlen_b32_hq32_hkv8_d128_p64_l512to4096",
+                        "b128_hq32_hkv8_d128_p16_l8192_bf16",
+                        "longctx_b4_hq16_hkv4_d256_p128_l32768_peaked",
+                        "fp8_verify_b64_q4_hq64_hkv8_d128_p128_w4096"}
+    for name, e in wls.items():
+        for k in ("ms_per_step", "tokens_per_s", "gb_s", "frac_of_copy", "frac_of_8tbs_spec",
+                  "kernel", "splits", "l2", "clocks", "avg_launch_ms",
+                  "algorithmic_bytes_per_step", "cpu_baseline"):
+            assert k in e, (name, k)
+        assert e["gb_s"] == pytest.approx(
+            e["algorithmic_bytes_per_step"] / (e["avg_launch_ms"] / 1e3) / 1e9, rel=1e-9)
+        assert e["frac_of_copy"] == pytest.approx(e["gb_s"] / rf["peak"], rel=1e-9)
+        assert e["tokens_per_s"] == pytest.approx(
+            e["batch"] * e["q_len"] / (e["ms_per_step"] / 1e3), rel=1e-6)
+        assert e["cpu_baseline"]["kind"] == "oracle" and e["cpu_baseline"]["value"] > 0
+        if name.startswith("tiny"):
+            assert e["l2"].startswith("flushed")
+        elif name.startswith("b128"):
+            assert e["l2"].startswith("no flush")
+        else:
+            assert e["l2"].startswith("rotating")
+    top = wls[cfg["workload"]]
+    assert top["top_level"] and top["ms_per_step"] == d["ms_per_step"]
