@@ -30,6 +30,8 @@
  *  - query head h reads kv head h / (num_q_heads / num_kv_heads).
  *  - KV pools are laid out [num_pages, num_kv_heads, page_size, head_dim].
  *  - FP8: element value = e4m3 code * kv_scale, one scale shared by K and V.
+ *  - NVFP4: element value = e2m1 code * e4m3 block scale * kv_scale, blocks
+ *    of 16 consecutive elements of a token row, kv_scale shared by K and V.
  *  - a row that sees no key gets out = 0 and lse = -inf.
  *
  * All entry points return a status and never abort or throw. Device work is
@@ -55,11 +57,20 @@ extern "C" {
 /* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
 typedef struct CUstream_st* pda_stream_t;
 
-#define PDA_ABI_VERSION 2
+#define PDA_ABI_VERSION 3
 
 typedef enum {
   PDA_KV_BF16 = 0,      /* K/V elements are bfloat16 */
-  PDA_KV_FP8_E4M3 = 1   /* K/V elements are FP8 E4M3 codes (uint8) */
+  PDA_KV_FP8_E4M3 = 1,  /* K/V elements are FP8 E4M3 codes (uint8) */
+  PDA_KV_NVFP4 = 2      /* K/V elements are NVFP4: FP4 E2M1 codes, two per byte
+                           (even element in the low nibble), with one E4M3
+                           scale per 16 consecutive elements of a row in
+                           separate scale pools (pda_params.k_scales /
+                           v_scales): value = e2m1 * e4m3 scale * kv_scale.
+                           "b12x 0.30.0, Kernel inventory": NVFP4
+                           (float4_e2m1fn) with E4M3 scales per 16 elements;
+                           "sglang profiler skill, fuse-overlap catalog": FP4
+                           paged KV caches. */
 } pda_kv_dtype;
 
 typedef enum {
@@ -105,7 +116,7 @@ typedef struct {
   int32_t causal_offset;    /* PDA_CAUSAL_OFF, PDA_CAUSAL_BOTTOM_RIGHT, or >= 0 */
   int32_t window;           /* <= 0 off; else keys j >= pos - window + 1 */
   int32_t kv_dtype;         /* pda_kv_dtype */
-  float kv_scale;           /* FP8 only: value = code * kv_scale (> 0) */
+  float kv_scale;           /* FP8 / NVFP4: value = code [* block scale] * kv_scale (> 0) */
   int32_t max_kv_len;       /* host hint, >= every kv_lens[b]; 0 -> max_pages_per_seq * P.
                                Used only to choose the split count. */
   int32_t num_splits;       /* 0 -> heuristic; > 0 forces this many KV splits */
@@ -118,6 +129,9 @@ typedef struct {
                                exp(sinks[h]) joins the softmax denominator and adds
                                no value; a row with no visible key then gets
                                out = 0, lse = sinks[h]. NULL: no sink. */
+  const void* k_scales;     /* NVFP4 only: device uint8 E4M3 block scales of K,
+                               [num_pages, Hkv, P, D/16], 16-byte aligned */
+  const void* v_scales;     /* NVFP4 only: the same for V. Ignored otherwise. */
 } pda_params;
 
 /*
@@ -125,7 +139,9 @@ typedef struct {
  *
  * q           device, bf16 [B, q_len, Hq, D], contiguous.
  * k_pages     device, [num_pages, Hkv, P, D] of bf16 (PDA_KV_BF16) or uint8
- * v_pages     e4m3 codes (PDA_KV_FP8_E4M3), contiguous.
+ * v_pages     e4m3 codes (PDA_KV_FP8_E4M3), or [num_pages, Hkv, P, D/2] of
+ *             packed e2m1 codes (PDA_KV_NVFP4, with params->k_scales and
+ *             v_scales), contiguous.
  * page_table  device, int32 [B, max_pages_per_seq]; entry t of row b is the
  *             pool page holding keys [t*P, (t+1)*P) of sequence b. Entries
  *             past ceil(kv_lens[b] / P) are never read (may hold -1).
@@ -153,7 +169,13 @@ typedef struct {
  * a kernel reads was written earlier in the same call. If params->workspace is NULL the library
  * uses a grow-only buffer it owns, one per device, shared by every call on
  * that device: calls that may overlap on different streams must pass their
- * own workspace (the same holds for a caller workspace).
+ * own workspace (the same holds for a caller workspace). A call that needs
+ * more than that buffer holds grows it in stream order on `stream`: the old
+ * buffer is released with cudaFreeAsync and the new one taken with
+ * cudaMallocAsync (the device's default memory pool); neither synchronises
+ * the device. During stream capture the buffer cannot grow: such a call
+ * returns PDA_ERR_WORKSPACE, so make one call with the largest params before
+ * capturing, or pass a workspace.
  *
  * Errors: invalid sizes or pointers return before any device work. A page
  * id >= num_pages or < 0 met on the device is never dereferenced; the kernel
@@ -174,24 +196,28 @@ PDA_API pda_status paged_decode_attn(const void* q, const void* k_pages,
  * device, and that cannot hand the library a workspace either.
  *
  * Same arguments and results as paged_decode_attn, except that
- * params->workspace and params->workspace_bytes are ignored: the split-KV
- * partials live in a fixed array of PDA_NO_ALLOC_WORKSPACE_BYTES compiled
- * into the library, which every device that loads the library holds until
- * the process exits. The call allocates nothing (no cudaMalloc, cudaFree or
- * allocating library routine).
+ * params->workspace and params->workspace_bytes are ignored: the call's
+ * whole workspace (the tensor-core kernel's counter header, its work-queue
+ * order and FP8 Q operand images, and the split-KV partials) lives in a
+ * fixed array of PDA_NO_ALLOC_WORKSPACE_BYTES compiled into the library,
+ * which every device that loads the library holds until the process exits.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine), and never uses the library-owned buffer of paged_decode_attn.
  *
- * Limit: if the partials of the chosen (or forced) split count need more
- * than PDA_NO_ALLOC_WORKSPACE_BYTES (see paged_decode_attn_workspace_bytes),
- * the call returns PDA_ERR_WORKSPACE before any device work.
+ * Limit: if paged_decode_attn_workspace_bytes(params) (the workspace of the
+ * chosen or forced split count and kernel) is more than
+ * PDA_NO_ALLOC_WORKSPACE_BYTES, the call returns PDA_ERR_WORKSPACE before
+ * any device work.
  *
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture.
  *
  * Sharing: all calls on a device use the same array, which keeps the last
- * call's partials. Nothing in it needs clearing (every slot a call reads was
- * written earlier in that call), but calls that overlap on the GPU (on
- * different streams) race on it: serialise them.
+ * call's contents. Nothing in it needs clearing by the caller (the
+ * tensor-core kernel's prologue zeroes its counters on every call, and every
+ * partial slot a call reads was written earlier in that call), but calls
+ * that overlap on the GPU (on different streams) race on it: serialise them.
  */
 #define PDA_NO_ALLOC_WORKSPACE_BYTES (16u * 1024u * 1024u)
 
@@ -204,12 +230,18 @@ PDA_API pda_status paged_decode_attn_no_alloc(const void* q, const void* k_pages
 
 /* Bytes of workspace paged_decode_attn needs for these params with the
  * split count it would choose (0 for the CUDA-core kernel when it would not
- * split). SIZE_MAX if the params are invalid. */
+ * split). SIZE_MAX if the params are invalid. The counterpart of
+ * alloc_split_partials ("AstrAI commit log,
+ * attn_paged_decode_split_kv_mma.cuh": split partials sized per call and
+ * never cleared). params->max_kv_len, the host's bound on the sequence
+ * lengths, takes the place of a separate length argument. */
 PDA_API size_t paged_decode_attn_workspace_bytes(const pda_params* params);
 
 /* The split count paged_decode_attn would use for these params on a device
- * with num_sms SMs (host-only; the heuristic of the split planner). Returns
- * a value >= 1, or 0 if params are invalid. */
+ * with num_sms SMs (host-only; the heuristic of the split planner, the
+ * counterpart of compute_num_splits in "AstrAI commit log,
+ * attn_paged_decode_split_kv_mma.cuh", driven by batch x kv heads against
+ * the SM count). Returns a value >= 1, or 0 if params are invalid. */
 PDA_API int32_t pda_choose_num_splits(const pda_params* params, int32_t num_sms);
 
 /*
@@ -246,7 +278,11 @@ typedef struct {
   int32_t max_pages_per_seq; /* row stride of page_table */
   int32_t num_pages;         /* pages in each pool; page ids must be < this */
   int32_t kv_dtype;          /* pda_kv_dtype of the pools */
-  float kv_scale;            /* FP8 only: code = e4m3(x / kv_scale) (> 0) */
+  float kv_scale;            /* FP8: code = e4m3(x / kv_scale); NVFP4: the per-tensor
+                                scale of the block rule below (> 0) */
+  void* k_scales;            /* NVFP4 only: device uint8 [num_pages, Hkv, P, D/16]
+                                block-scale pools, written for the appended rows */
+  void* v_scales;
 } pda_append_params;
 
 /*
@@ -268,7 +304,13 @@ typedef struct {
  * bf16 pools receive the bits unchanged. FP8 pools receive, per element, the
  * e4m3 code nearest to the fp32 quotient x / kv_scale (IEEE division), ties
  * to even, saturated to +-448 (NaN stays NaN): the encoding the decode call
- * inverts with the same kv_scale.
+ * inverts with the same kv_scale. NVFP4 pools receive, per block of 16
+ * elements of a row ("b12x 0.30.0, Kernel inventory", BF16-to-FP4 TMA
+ * quantization row: packed NVFP4 plus scale tiles; "sglang profiler skill,
+ * fuse-overlap catalog", fused BF16 to FP4 quant + paged KV write row), all
+ * in fp32 with nearest-even rounding and saturation: q = x / kv_scale,
+ * block scale = e4m3(max |q| / 6), code = e2m1(q / block scale) (a block
+ * whose scale is zero stores +0 codes); NaN inputs give unspecified codes.
  *
  * Errors: invalid params or pointers return before any device work
  * (PDA_ERR_INVALID_ARG / _UNSUPPORTED / _MISALIGNED). A position past
@@ -282,7 +324,9 @@ PDA_API pda_status paged_kv_append(const void* k_new, const void* v_new,
                                    void* v_pages, pda_stream_t stream);
 
 /* Which split kernel paged_decode_attn would launch for these params
- * (host-only; the planner's choice):
+ * (host-only; the planner's choice between the two variants that "AstrAI
+ * commit log, attn_paged_decode_split_kv_mma.cuh" describes: the scalar
+ * variant and the tensor-core head-packing variant):
  *   PDA_KERNEL_SPLIT_TMA  tensor-core kernel (2D TMA tiles of 128 tokens,
  *                         tcgen05 MMAs with TMEM accumulators): head_dim 128
  *                         with bf16 K/V and at most 8 packed rows per kv head
@@ -310,7 +354,10 @@ PDA_API pda_status pda_hbm_read_probe(const void* buf, size_t bytes, uint64_t* s
 /* Human-readable name of a status. Never NULL. */
 PDA_API const char* pda_status_string(pda_status status);
 
-/* Synchronises `stream`, then reads and clears the current device's error
+/* The pages have no counterpart to this entry point: it reports what the
+ * kernels' in-bounds checks found (a debug read, the one call that
+ * synchronises).
+ * Synchronises `stream`, then reads and clears the current device's error
  * word: the first error a kernel recorded since the last read
  * (PDA_ERR_BAD_PAGE, PDA_ERR_TIMEOUT, or PDA_ERR_UNSUPPORTED if a kernel met
  * a launch condition it cannot handle), PDA_OK otherwise (PDA_ERR_CUDA if the

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(PKG, "libpaged_decode_attn.so")
 
 PDA_KV_BF16 = 0
 PDA_KV_FP8_E4M3 = 1
+PDA_KV_NVFP4 = 2
 PDA_CAUSAL_OFF = -1
 PDA_CAUSAL_BOTTOM_RIGHT = -2
 PDA_FLAG_NO_PDL = 1
@@ -24,7 +25,7 @@ PDA_FLAG_TENSOR_CORES = 2
 PDA_FLAG_CUDA_CORES = 4
 PDA_FLAG_FUSED_MERGE = 8
 PDA_FLAG_NATIVE_FP8_QK = 16
-# Size of the library's fixed partials array used by paged_decode_attn_no_alloc.
+# Size of the library's fixed workspace array used by paged_decode_attn_no_alloc.
 PDA_NO_ALLOC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 STATUS = {
@@ -64,6 +65,8 @@ class PdaAppendParams(ctypes.Structure):
         ("num_pages", ctypes.c_int32),
         ("kv_dtype", ctypes.c_int32),
         ("kv_scale", ctypes.c_float),
+        ("k_scales", ctypes.c_void_p),
+        ("v_scales", ctypes.c_void_p),
     ]
 
 
@@ -91,6 +94,8 @@ class PdaParams(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("num_splits_out", ctypes.POINTER(ctypes.c_int32)),
         ("sinks", ctypes.c_void_p),
+        ("k_scales", ctypes.c_void_p),
+        ("v_scales", ctypes.c_void_p),
     ]
 
 
@@ -191,36 +196,61 @@ def _stream_handle(stream) -> Optional[int]:
     return s.cuda_stream or None
 
 
+def _params_for(q, k_pages, v_pages, page_table, kv_lens, k_scales, v_scales, **kw):
+    """pda_params for CUDA tensors (checks they are contiguous CUDA tensors);
+    the KV dtype follows the pools: bf16, uint8 e4m3 codes, or uint8 NVFP4
+    codes when block-scale pools are given."""
+    import torch
+    B, q_len, Hq, D = q.shape
+    for t in (q, k_pages, v_pages, page_table, kv_lens):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("all inputs must be contiguous CUDA tensors")
+    if k_scales is not None or v_scales is not None:
+        for t in (k_scales, v_scales):
+            if t is None or not t.is_cuda or not t.is_contiguous() or t.dtype != torch.uint8:
+                raise ValueError("k_scales and v_scales must be contiguous uint8 CUDA tensors")
+        kv_dtype = PDA_KV_NVFP4
+    else:
+        kv_dtype = PDA_KV_FP8_E4M3 if k_pages.dtype == torch.uint8 else PDA_KV_BF16
+    params = make_params(
+        batch=B, q_len=q_len, num_q_heads=Hq, head_dim=D, page_size=k_pages.shape[2],
+        max_pages_per_seq=page_table.shape[1], num_pages=k_pages.shape[0],
+        kv_dtype=kv_dtype, **kw)
+    if kv_dtype == PDA_KV_NVFP4:
+        params.k_scales = k_scales.data_ptr()
+        params.v_scales = v_scales.data_ptr()
+    return params
+
+
 def paged_decode_attn(q, k_pages, v_pages, page_table, kv_lens, *, num_kv_heads,
                       scale, causal_offset=PDA_CAUSAL_OFF, window=0, kv_scale=1.0,
                       max_kv_len=0, num_splits=0, flags=0, out=None, lse=None,
-                      workspace=None, stream=None, with_lse=True, sinks=None):
+                      workspace=None, stream=None, with_lse=True, sinks=None,
+                      library_workspace=False, k_scales=None, v_scales=None):
     """Run the library on CUDA tensors; returns (out, lse, num_splits_used).
 
     q [B, q_len, Hq, D] bf16; k/v_pages [num_pages, Hkv, P, D] bf16 or uint8
-    (e4m3 codes); page_table int32 [B, max_pages]; kv_lens int32 [B];
+    (e4m3 codes), or with k_scales / v_scales (uint8 [num_pages, Hkv, P,
+    D/16] e4m3 block scales) uint8 [num_pages, Hkv, P, D/2] NVFP4 codes;
+    page_table int32 [B, max_pages]; kv_lens int32 [B];
     sinks: optional float32 CUDA tensor [Hq] of attention-sink logits.
     ``workspace``: a CUDA uint8 tensor (any contents; reusable across calls),
     or None to let the binding allocate exactly what the call needs.
+    ``library_workspace``: pass no workspace, so the library uses (and grows
+    in stream order) the buffer it owns on the device.
     """
     import torch
     lib = load()
     B, q_len, Hq, D = q.shape
-    kv_dtype = PDA_KV_FP8_E4M3 if k_pages.dtype == torch.uint8 else PDA_KV_BF16
-    for t in (q, k_pages, v_pages, page_table, kv_lens):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("all inputs must be contiguous CUDA tensors")
-    params = make_params(
-        batch=B, q_len=q_len, num_q_heads=Hq, num_kv_heads=num_kv_heads, head_dim=D,
-        page_size=k_pages.shape[2], max_pages_per_seq=page_table.shape[1],
-        num_pages=k_pages.shape[0], scale=scale, causal_offset=causal_offset,
-        window=window, kv_dtype=kv_dtype, kv_scale=kv_scale, max_kv_len=max_kv_len,
-        num_splits=num_splits, flags=flags)
+    params = _params_for(q, k_pages, v_pages, page_table, kv_lens, k_scales, v_scales,
+                         num_kv_heads=num_kv_heads, scale=scale, causal_offset=causal_offset,
+                         window=window, kv_scale=kv_scale, max_kv_len=max_kv_len,
+                         num_splits=num_splits, flags=flags)
     if out is None:
         out = torch.empty((B, q_len, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None and with_lse:
         lse = torch.empty((B, q_len, Hq), dtype=torch.float32, device=q.device)
-    if workspace is None:
+    if workspace is None and not library_workspace:
         need = lib.paged_decode_attn_workspace_bytes(ctypes.byref(params))
         if need == ctypes.c_size_t(-1).value:
             raise PdaError(1, "paged_decode_attn_workspace_bytes")
@@ -246,24 +276,30 @@ def paged_decode_attn(q, k_pages, v_pages, page_table, kv_lens, *, num_kv_heads,
 def paged_decode_attn_no_alloc(q, k_pages, v_pages, page_table, kv_lens, *,
                                num_kv_heads, scale, causal_offset=PDA_CAUSAL_OFF,
                                window=0, kv_scale=1.0, max_kv_len=0, num_splits=0,
-                               flags=0, out=None, lse=None, stream=None):
-    """The allocation-free entry point: split partials go to the library's
-    fixed device array instead of a workspace (see the C header). ``out`` and
-    ``lse`` are allocated here by torch only when the caller passes None."""
+                               flags=0, out=None, lse=None, stream=None, sinks=None,
+                               k_scales=None, v_scales=None):
+    """The allocation-free entry point: the call's whole workspace goes to
+    the library's fixed device array (see the C header). Same arguments as
+    paged_decode_attn minus ``workspace``. ``out`` and ``lse`` are allocated
+    here by torch only when the caller passes None."""
     import torch
     lib = load()
     B, q_len, Hq, D = q.shape
-    kv_dtype = PDA_KV_FP8_E4M3 if k_pages.dtype == torch.uint8 else PDA_KV_BF16
-    params = make_params(
-        batch=B, q_len=q_len, num_q_heads=Hq, num_kv_heads=num_kv_heads, head_dim=D,
-        page_size=k_pages.shape[2], max_pages_per_seq=page_table.shape[1],
-        num_pages=k_pages.shape[0], scale=scale, causal_offset=causal_offset,
-        window=window, kv_dtype=kv_dtype, kv_scale=kv_scale, max_kv_len=max_kv_len,
-        num_splits=num_splits, flags=flags)
+    params = _params_for(q, k_pages, v_pages, page_table, kv_lens, k_scales, v_scales,
+                         num_kv_heads=num_kv_heads, scale=scale, causal_offset=causal_offset,
+                         window=window, kv_scale=kv_scale, max_kv_len=max_kv_len,
+                         num_splits=num_splits, flags=flags)
     if out is None:
         out = torch.empty((B, q_len, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, q_len, Hq), dtype=torch.float32, device=q.device)
+    for t in (out, lse):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float32:
+            raise ValueError("out and lse must be contiguous float32 CUDA tensors")
+    if sinks is not None:
+        if not (sinks.is_cuda and sinks.dtype == torch.float32 and sinks.numel() == Hq):
+            raise ValueError("sinks must be a float32 CUDA tensor of num_q_heads entries")
+        params.sinks = sinks.data_ptr()
     used = ctypes.c_int32(0)
     params.num_splits_out = ctypes.pointer(used)
     st = lib.paged_decode_attn_no_alloc(
@@ -275,18 +311,23 @@ def paged_decode_attn_no_alloc(q, k_pages, v_pages, page_table, kv_lens, *,
 
 
 def paged_kv_append(k_new, v_new, page_table, kv_lens, k_pages, v_pages, *, kv_scale=1.0,
-                    stream=None):
+                    stream=None, k_scales=None, v_scales=None):
     """Write new K/V rows (bf16 [B, num_new, Hkv, D]) into the pools at
     positions kv_lens[b] + t (kv_lens is not advanced). Pools of uint8 are
-    e4m3 codes quantised with kv_scale; bf16 pools get the bits."""
+    e4m3 codes quantised with kv_scale, or, with k_scales / v_scales (uint8
+    block-scale pools), NVFP4 codes; bf16 pools get the bits."""
     import torch
     B, T, Hkv, D = k_new.shape
     kv_dtype = PDA_KV_FP8_E4M3 if k_pages.dtype == torch.uint8 else PDA_KV_BF16
-    for t_ in (k_new, v_new, page_table, kv_lens, k_pages, v_pages):
-        if not t_.is_cuda or not t_.is_contiguous():
+    tensors = [k_new, v_new, page_table, kv_lens, k_pages, v_pages]
+    if k_scales is not None or v_scales is not None:
+        kv_dtype = PDA_KV_NVFP4
+        tensors += [k_scales, v_scales]
+    for t_ in tensors:
+        if t_ is None or not t_.is_cuda or not t_.is_contiguous():
             raise ValueError("all inputs must be contiguous CUDA tensors")
     p = PdaAppendParams(B, T, Hkv, D, k_pages.shape[2], page_table.shape[1], k_pages.shape[0],
-                        kv_dtype, kv_scale)
+                        kv_dtype, kv_scale, _ptr(k_scales), _ptr(v_scales))
     st = load().paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(page_table), _ptr(kv_lens),
                                 ctypes.byref(p), _ptr(k_pages), _ptr(v_pages),
                                 _stream_handle(stream))

@@ -95,6 +95,7 @@ bool pool_rows_fit(const pda_params* p) {
 // The flags force either kernel.
 bool use_tensor_cores(const pda_params* p, int M) {
   if (p->head_dim != 128 || p->page_size < 8 || !pool_rows_fit(p)) return false;
+  if (p->kv_dtype == PDA_KV_NVFP4) return false;  // the CUDA-core kernel decodes NVFP4
   if (p->flags & PDA_FLAG_CUDA_CORES) return false;
   if (p->flags & PDA_FLAG_TENSOR_CORES) return true;
   return p->kv_dtype == PDA_KV_FP8_E4M3 ? M > 8 : M <= 8;
@@ -109,8 +110,10 @@ pda_status validate(const pda_params* p) {
     return PDA_ERR_INVALID_ARG;
   if (!(p->scale > 0.f) || !std::isfinite(p->scale)) return PDA_ERR_INVALID_ARG;
   if (p->causal_offset < PDA_CAUSAL_BOTTOM_RIGHT) return PDA_ERR_INVALID_ARG;
-  if (p->kv_dtype != PDA_KV_BF16 && p->kv_dtype != PDA_KV_FP8_E4M3) return PDA_ERR_INVALID_ARG;
-  if (p->kv_dtype == PDA_KV_FP8_E4M3 && (!(p->kv_scale > 0.f) || !std::isfinite(p->kv_scale)))
+  if (p->kv_dtype != PDA_KV_BF16 && p->kv_dtype != PDA_KV_FP8_E4M3 &&
+      p->kv_dtype != PDA_KV_NVFP4)
+    return PDA_ERR_INVALID_ARG;
+  if (p->kv_dtype != PDA_KV_BF16 && (!(p->kv_scale > 0.f) || !std::isfinite(p->kv_scale)))
     return PDA_ERR_INVALID_ARG;
   if (p->max_kv_len < 0 || p->num_splits < 0) return PDA_ERR_INVALID_ARG;
   if ((long long)p->max_pages_per_seq * p->page_size > INT_MAX) return PDA_ERR_INVALID_ARG;
@@ -126,7 +129,7 @@ Plan make_plan(const pda_params* p) {
   Plan pl{};
   pl.G = p->num_q_heads / p->num_kv_heads;
   pl.M = pl.G * p->q_len;
-  pl.elt = p->kv_dtype == PDA_KV_BF16 ? 2 : 1;
+  pl.elt = p->kv_dtype == PDA_KV_BF16 ? 2 : 1;  // NVFP4: codes are half a byte (see below)
   pl.rows = (long long)p->batch * p->q_len * p->num_q_heads;
   pl.tc = use_tensor_cores(p, pl.M);
   if (pl.tc) {
@@ -308,6 +311,9 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
     return PDA_OK;
   }
   if (!q || !k_pages || !v_pages || !page_table || !kv_lens || !out) return PDA_ERR_INVALID_ARG;
+  const bool nvfp4 = p.kv_dtype == PDA_KV_NVFP4;
+  if (nvfp4 && (!p.k_scales || !p.v_scales)) return PDA_ERR_INVALID_ARG;
+  if (nvfp4 && (!aligned(p.k_scales, 16) || !aligned(p.v_scales, 16))) return PDA_ERR_MISALIGNED;
   if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
       !aligned(page_table, 4) || !aligned(kv_lens, 4) || (lse && !aligned(lse, 4)) ||
       (p.sinks && !aligned(p.sinks, 4)))
@@ -349,10 +355,18 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   a.window = p.window;
   const float log2e = 1.4426950408889634f;
   const bool fp8 = p.kv_dtype == PDA_KV_FP8_E4M3;
-  a.qk_scale_log2 = p.scale * log2e * (fp8 ? p.kv_scale : 1.f);
-  a.v_scale = fp8 ? p.kv_scale : 1.f;
-  a.head_stride = (long long)p.page_size * p.head_dim * pl.elt;
+  const bool scaled = p.kv_dtype != PDA_KV_BF16;  // FP8 and NVFP4 carry kv_scale
+  a.qk_scale_log2 = p.scale * log2e * (scaled ? p.kv_scale : 1.f);
+  a.v_scale = scaled ? p.kv_scale : 1.f;
+  a.head_stride = nvfp4 ? (long long)p.page_size * p.head_dim / 2
+                        : (long long)p.page_size * p.head_dim * pl.elt;
   a.page_stride = a.head_stride * p.num_kv_heads;
+  if (nvfp4) {
+    a.k_scales = static_cast<const uint8_t*>(p.k_scales);
+    a.v_scales = static_cast<const uint8_t*>(p.v_scales);
+    a.sc_head_stride = (long long)p.page_size * p.head_dim / 16;
+    a.sc_page_stride = a.sc_head_stride * p.num_kv_heads;
+  }
 
   const WsLayout wl = ws_layout(&p, pl, splits);
   if (wl.total > 0) {
@@ -360,13 +374,23 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
     if (ws == nullptr) {
       std::lock_guard<std::mutex> lock(g_mu);
       if (dev->ws_bytes < wl.total) {
-        if (dev->ws) cudaFree(dev->ws);  // synchronises the device
+        // Grow stream-ordered: the old buffer is released after the work
+        // already queued on `stream`, the new one is ready for the work
+        // queued next, and neither step synchronises the device. A call
+        // being captured into a CUDA graph cannot grow the buffer (the
+        // allocation would belong to the graph).
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return PDA_ERR_CUDA;
+        if (cap != cudaStreamCaptureStatusNone) return PDA_ERR_WORKSPACE;
+        if (dev->ws && cudaFreeAsync(dev->ws, stream) != cudaSuccess) return PDA_ERR_CUDA;
         dev->ws = nullptr;
         dev->ws_bytes = 0;
-        if (cudaMalloc(&dev->ws, wl.total) != cudaSuccess) {
-          dev->ws = nullptr;
+        void* fresh = nullptr;
+        if (cudaMallocAsync(&fresh, wl.total, stream) != cudaSuccess) {
+          (void)cudaGetLastError();
           return PDA_ERR_WORKSPACE;
         }
+        dev->ws = fresh;
         dev->ws_bytes = wl.total;
       }
       ws = dev->ws;
@@ -390,7 +414,7 @@ pda_status paged_decode_attn(const void* q, const void* k_pages, const void* v_p
   }
 
   cudaError_t e;
-  const int kv = fp8 ? 1 : 0;
+  const int kv = nvfp4 ? 2 : (fp8 ? 1 : 0);
   if (pl.tc) {
     // persistent: at most one CTA per SM, items from the work queue; the
     // split that finishes last for a group of rows merges it (no merge launch)

@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -187,6 +188,22 @@ __device__ __forceinline__ f32x2 e4m3x2_to_f2(uint32_t h16) {
       __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(h16 & 0xFFFFu), __NV_E4M3);
   const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
   return f2_pack(f.x, f.y);
+}
+
+// Two e2m1 codes (one byte, first element in the low nibble) -> the fp32
+// pair (exact: e2m1 -> f16 -> f32).
+__device__ __forceinline__ f32x2 e2m1x2_to_f2(uint32_t byte) {
+  const __half2_raw hr =
+      __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte & 0xFFu), __NV_E2M1);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+  return f2_pack(f.x, f.y);
+}
+
+// One e4m3 code -> float (exact).
+__device__ __forceinline__ float e4m3_code_to_f32(uint32_t code) {
+  const __half_raw h =
+      __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code & 0xFFu), __NV_E4M3);
+  return __half2float(*reinterpret_cast<const __half*>(&h));
 }
 
 }  // namespace pda

@@ -6,7 +6,8 @@
 // multi-stage copy pipeline keeping STAGES-1 tiles in flight; predicated
 // partial tiles; split partials written without a memset), "b12x 0.30.0,
 // Kernel inventory, Attention table, Paged attention row" (bf16 and
-// FP8-E4M3 KV, sliding window, GQA, split-KV or direct output).
+// FP8-E4M3 KV, sliding window, GQA, split-KV or direct output) and the same
+// inventory's NVFP4 rows (float4_e2m1fn with E4M3 scales per 16 elements).
 //
 // B200 design:
 //  * One CTA per (row tile, split, kv head, sequence). The CTA's key range is
@@ -21,13 +22,15 @@
 //    A page id outside [0, num_pages) is recorded as an error and replaced by
 //    page 0, so no access ever leaves the pool.
 //  * Lane layout: a token's D elements are split over LPT = D/8 lanes, 8
-//    elements (one 16-byte bf16 or 8-byte e4m3 load) per lane; TPI = 32/LPT
+//    elements (one 16-byte bf16, 8-byte e4m3 or 4-byte NVFP4 load, plus the
+//    block's e4m3 scale byte) per lane; TPI = 32/LPT
 //    tokens are read per warp instruction (a warp reads 512 contiguous bytes
 //    for bf16, conflict-free). Q sits in registers, pre-scaled by
-//    scale*log2(e) (and kv_scale for FP8), for the lane's 8 elements of each
+//    scale*log2(e) (and kv_scale for FP8 / NVFP4), for the lane's 8 elements of each
 //    of the M_T rows.
 //  * Arithmetic runs on packed fp32 pairs (fma/mul.rn.f32x2: two FMAs per
-//    issue slot); bf16 and e4m3 elements convert straight into pairs.
+//    issue slot); bf16, e4m3 and e2m1 (times its block scale, exact)
+//    elements convert straight into pairs.
 //  * Scores: 8*M_T partial dot products per lane per group of 8 tokens are
 //    summed over the LPT lanes of a token with a reduce-scatter butterfly
 //    (each step halves the values a lane carries), so a score costs about one
@@ -56,8 +59,12 @@ constexpr int kMergeCtrPerGroup = 4;
 
 struct SplitArgs {
   const uint16_t* q;         // bf16 bits [B, Lq, Hq, D]
-  const uint8_t* k_pages;    // pool bytes [num_pages, Hkv, P, D]
+  const uint8_t* k_pages;    // pool bytes [num_pages, Hkv, P, D] (NVFP4: D/2)
   const uint8_t* v_pages;
+  const uint8_t* k_scales;   // NVFP4: e4m3 block scales [num_pages, Hkv, P, D/16]
+  const uint8_t* v_scales;
+  long long sc_page_stride;  // NVFP4: bytes per page / per (page, head) block
+  long long sc_head_stride;  //   of the scale pools
   const int32_t* page_table; // [B, max_pages]
   const int32_t* kv_lens;    // [B]
   float* out;                // [B, Lq, Hq, D]       (num_splits == 1)
@@ -70,10 +77,10 @@ struct SplitArgs {
   int tile_shift;            // log2(page_size / TW): tiles per page
   int num_splits, row_tiles;
   int causal_offset, window;
-  float qk_scale_log2;       // scale * log2(e) [* kv_scale for FP8]
-  float v_scale;             // 1, or kv_scale for FP8
-  long long page_stride;     // bytes per page: Hkv * P * D * elt
-  long long head_stride;     // bytes per (page, head) block: P * D * elt
+  float qk_scale_log2;       // scale * log2(e) [* kv_scale for FP8 / NVFP4]
+  float v_scale;             // 1, or kv_scale for FP8 / NVFP4
+  long long page_stride;     // bytes per page of the code pool: Hkv * P * D * elt
+  long long head_stride;     // bytes per (page, head) block: P * D * elt (NVFP4: elt 1/2)
   // persistent tensor-core kernel only (prepared by its prologue kernel,
   // which runs just before it on the same stream):
   int* sched;                // [0] next work item
@@ -87,9 +94,11 @@ struct SplitArgs {
   int fused_merge;           // 1: the last split of a group merges it in-kernel
 };
 
+// KV: 0 bf16, 1 e4m3, 2 NVFP4 (e2m1 codes two per byte + an e4m3 scale per
+// 16 elements; a stage then holds K codes, K scales, V codes, V scales).
 template <int D, int KV, int MT, int TW, int NW, int STAGES>
 struct FmaCfg {
-  static constexpr int ELT = KV == 0 ? 2 : 1;
+  static constexpr int ELT = KV == 0 ? 2 : 1;  // bytes per element (KV 0, 1)
   static constexpr int CH = 8;             // elements per lane chunk
   static constexpr int LPT = D / CH;       // lanes per token
   static constexpr int TPI = 32 / LPT;     // tokens per warp instruction
@@ -101,8 +110,10 @@ struct FmaCfg {
   static constexpr int NFOLD = NVF > MT ? MT : NVF;
   static constexpr int RED_LO =
       NV >= LPT ? (NVF >= MT ? 1 : MT / NVF) : (LPT / NV) * MT;
-  static constexpr int TILE_BYTES = TW * D * ELT;
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int TILE_BYTES = KV == 2 ? TW * D / 2 : TW * D * ELT;  // K or V codes
+  static constexpr int SC_BYTES = KV == 2 ? TW * D / 16 : 0;              // their block scales
+  static constexpr int HALF_STAGE = TILE_BYTES + SC_BYTES;                // K (or V) part
+  static constexpr int STAGE_BYTES = 2 * HALF_STAGE;
   static constexpr int PBUF_FLOATS = TW * MT * 2;  // (p, p) pairs
   static constexpr int WARP_SMEM_RAW =
       STAGES * STAGE_BYTES + 32 /*mbarriers*/ + PBUF_FLOATS * 4 + 64 /*alpha pairs*/;
@@ -119,7 +130,8 @@ struct FmaCfg {
   static_assert(D % 64 == 0 && D <= 256, "head_dim");
   static_assert(TW % TPI == 0 && NTOK >= 1, "tile");
   static_assert(STAGES <= 4, "mbarrier area holds 4");
-  static_assert(TILE_BYTES % 16 == 0, "bulk copy size");
+  static_assert(TILE_BYTES % 16 == 0 && SC_BYTES % 16 == 0, "bulk copy size");
+  static_assert(KV != 2 || D % 16 == 0, "NVFP4 blocks of 16 elements");
 };
 
 // Visible key range [lo, hi) of a query row at index i (reading of the
@@ -159,6 +171,18 @@ __device__ __forceinline__ void reduce_scatter(float* v) {
       reduce_scatter<1, O / 2>(v);
     }
   }
+}
+
+// NVFP4: 8 consecutive elements of one token (4 code bytes) and the e4m3
+// scale of their block -> 4 fp32 pairs (exact: e2m1 * e4m3 has 5
+// significant bits).
+__device__ __forceinline__ void load_chunk_nvfp4(const uint8_t* codes, const uint8_t* scale,
+                                                 f32x2 (&f)[4]) {
+  const uint32_t c = *reinterpret_cast<const uint32_t*>(codes);
+  const float sc = e4m3_code_to_f32(*scale);
+  const f32x2 s2 = f2_pack(sc, sc);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f[k] = f2_mul(e2m1x2_to_f2(c >> (8 * k)), s2);
 }
 
 // 8 consecutive K or V elements of one token -> 4 fp32 pairs.
@@ -225,6 +249,8 @@ __global__ void __launch_bounds__(NW * 32, 1)
   const int32_t* pt_row = a.page_table + (long long)b * a.max_pages;
   const uint8_t* kbase_ptr = a.k_pages + (long long)kvh * a.head_stride;
   const uint8_t* vbase_ptr = a.v_pages + (long long)kvh * a.head_stride;
+  const uint8_t* ksc_ptr = KV == 2 ? a.k_scales + (long long)kvh * a.sc_head_stride : nullptr;
+  const uint8_t* vsc_ptr = KV == 2 ? a.v_scales + (long long)kvh * a.sc_head_stride : nullptr;
 
   // ---- barriers and page-id prefetch -------------------------------------
   if (lane == 0) {
@@ -257,12 +283,17 @@ __global__ void __launch_bounds__(NW * 32, 1)
     const int pid = __shfl_sync(FULL, pid_cur, n & 31);
     if (lane == 0) {
       const int s = n % STAGES;
-      const long long off = (long long)pid * a.page_stride +
-                            (long long)((kbase + n * NW) & tile_mask) * C::TILE_BYTES;
+      const long long tip = (long long)((kbase + n * NW) & tile_mask);  // tile in page
+      const long long off = (long long)pid * a.page_stride + tip * C::TILE_BYTES;
       uint8_t* dst = wbase + s * C::STAGE_BYTES;
       mbar_arrive_expect_tx(&mbar[s], C::STAGE_BYTES);
       bulk_g2s(dst, kbase_ptr + off, C::TILE_BYTES, &mbar[s]);
-      bulk_g2s(dst + C::TILE_BYTES, vbase_ptr + off, C::TILE_BYTES, &mbar[s]);
+      bulk_g2s(dst + C::HALF_STAGE, vbase_ptr + off, C::TILE_BYTES, &mbar[s]);
+      if constexpr (KV == 2) {
+        const long long soff = (long long)pid * a.sc_page_stride + tip * C::SC_BYTES;
+        bulk_g2s(dst + C::TILE_BYTES, ksc_ptr + soff, C::SC_BYTES, &mbar[s]);
+        bulk_g2s(dst + C::HALF_STAGE + C::TILE_BYTES, vsc_ptr + soff, C::SC_BYTES, &mbar[s]);
+      }
     }
   };
 
@@ -341,7 +372,14 @@ __global__ void __launch_bounds__(NW * 32, 1)
       break;
     }
     const uint8_t* kt = wbase + s * C::STAGE_BYTES;
-    const uint8_t* vt = kt + C::TILE_BYTES;
+    const uint8_t* vt = kt + C::HALF_STAGE;
+    // 8 elements of token `tok` from this lane's chunk, as 4 fp32 pairs
+    auto load_tok = [&](const uint8_t* tile, int tok, f32x2 (&f)[4]) {
+      if constexpr (KV == 2)
+        load_chunk_nvfp4(tile + (tok * D + d0) / 2, tile + C::TILE_BYTES + (tok * D + d0) / 16, f);
+      else
+        load_chunk2<KV>(tile + (tok * D + d0) * C::ELT, f);
+    };
     const int t0 = (kbase + n * NW) * TW;
     const bool clean = t0 >= lo_x && t0 + TW <= hi_x;
 
@@ -351,7 +389,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
     for (int it = 0; it < C::NTOK; ++it) {
       const int tok = (it ^ vmask_it) * C::TPI + grp;
       f32x2 kf[4];
-      load_chunk2<KV>(kt + (tok * D + d0) * C::ELT, kf);
+      load_tok(kt, tok, kf);
 #pragma unroll
       for (int r = 0; r < MT; ++r) {
         f32x2 s2 = f2_mul(qf[r][0], kf[0]);
@@ -439,7 +477,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
         pr[0] = f2_pack(p2.x, p2.y);
       }
       f32x2 vf[4];
-      load_chunk2<KV>(vt + (tok * D + d0) * C::ELT, vf);
+      load_tok(vt, tok, vf);
       if (!clean) {
         const int j = t0 + tok;
         if (j < lo_u || j >= hi_u) {

@@ -67,8 +67,10 @@ cudaError_t launch_for_dim(int kv, int mt, int tw, const SplitArgs& a,
   }
   if (kv == 0) {
     PDA_MT_CASES(0)
-  } else {
+  } else if (kv == 1) {
     PDA_MT_CASES(1)
+  } else {
+    PDA_MT_CASES(2)
   }
 #undef PDA_MT_CASES
 }

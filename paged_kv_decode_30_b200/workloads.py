@@ -114,6 +114,12 @@ FP8_VERIFY = Workload(
 
 ALL = {w.name: w for w in (TINY, VARLEN, HEADLINE, LONGCTX, FP8_VERIFY)}
 
+# The headline shape with an NVFP4 KV cache (a KV dtype beyond the five
+# workloads: the same sequences, 72 bytes per token row of K or V instead of
+# 256).
+NVFP4_HEADLINE = HEADLINE.with_(name="nvfp4_b128_hq32_hkv8_d128_p16_l8192", kv_dtype=KV_NVFP4)
+EXTRA = {NVFP4_HEADLINE.name: NVFP4_HEADLINE}
+
 
 def _draw_kv_lens(wl: Workload, gen: torch.Generator) -> torch.Tensor:
     kind = wl.kv_lens[0]
@@ -304,6 +310,12 @@ def encode_nvfp4(x: torch.Tensor, kv_scale: float):
     the even code, saturating at 6; +0 codes where the scale is zero).
     Returns (codes packed two per byte [..., D/2], scales [..., D/16])."""
     D = x.shape[-1]
+    rows = x.reshape(-1, D)
+    step = max(1, (1 << 24) // D)  # rows per chunk: bounded temporaries
+    if rows.shape[0] > step:
+        parts = [encode_nvfp4(rows[i:i + step], kv_scale) for i in range(0, rows.shape[0], step)]
+        return (torch.cat([p_[0] for p_ in parts]).reshape(*x.shape[:-1], D // 2),
+                torch.cat([p_[1] for p_ in parts]).reshape(*x.shape[:-1], D // NVFP4_BLOCK))
     q = x.float() / kv_scale
     blk = q.reshape(*q.shape[:-1], D // NVFP4_BLOCK, NVFP4_BLOCK)
     amax = blk.abs().amax(dim=-1)

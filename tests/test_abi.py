@@ -52,7 +52,7 @@ def test_only_c_abi_symbols_are_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.pda_abi_version() == 2
+    assert lib.pda_abi_version() == 3
     for code in range(8):
         assert B.status_string(code)
     assert B.status_string(99) == "unknown status"
@@ -78,7 +78,8 @@ def headline_params(**over):
     (dict(scale=0.0), 1),
     (dict(scale=float("nan")), 1),
     (dict(causal_offset=-3), 1),
-    (dict(kv_dtype=2), 1),
+    (dict(kv_dtype=3), 1),
+    (dict(kv_dtype=2, kv_scale=0.0), 1),
     (dict(kv_dtype=1, kv_scale=0.0), 1),
     (dict(num_pages=0), 1),
     (dict(max_pages_per_seq=0), 1),
@@ -244,3 +245,52 @@ def test_append_validation(lib):
     p = B.PdaAppendParams(2, 1, 2, 128, 16, 4, 8, B.PDA_KV_BF16, 1.0)
     assert lib.paged_kv_append((1 << 20) + 8, 1 << 20, 1 << 20, 1 << 20, ctypes.byref(p),
                                1 << 20, 1 << 20, None) == 3
+
+
+def test_binding_structs_match_the_header_layout(tmp_path):
+    """The ctypes mirrors of pda_params and pda_append_params have the C
+    header's size and field offsets (a C program compiled against the header
+    prints them)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    structs = {"pda_params": B.PdaParams, "pda_append_params": B.PdaAppendParams}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "paged_decode_attn.h"',
+             'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    got = {}
+    for line in out.splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_nvfp4_needs_aligned_scale_pools(lib):
+    ok = ctypes.c_void_p(1 << 20)
+    p = headline_params(kv_dtype=B.PDA_KV_NVFP4, kv_scale=0.01)
+    st = lib.paged_decode_attn(ok, ok, ok, ok, ok, ctypes.byref(p), ok, ok, None)
+    assert st == 1  # no block-scale pools
+    p.k_scales = (1 << 20) + 4
+    p.v_scales = 1 << 20
+    st = lib.paged_decode_attn(ok, ok, ok, ok, ok, ctypes.byref(p), ok, ok, None)
+    assert st == 3
+    a = B.PdaAppendParams(4, 1, 8, 128, 16, 8, 64, B.PDA_KV_NVFP4, 0.01, None, None)
+    st = lib.paged_kv_append(ok, ok, ok, ok, ctypes.byref(a), ok, ok, None)
+    assert st == 1
+    # the planner keeps NVFP4 on the CUDA-core kernel, whatever the flags
+    p = headline_params(kv_dtype=B.PDA_KV_NVFP4, kv_scale=0.01, flags=B.PDA_FLAG_TENSOR_CORES)
+    assert B.plan_kernel(p) == B.PDA_KERNEL_SPLIT_FMA

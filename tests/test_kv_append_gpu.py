@@ -29,38 +29,79 @@ def _case(seed, B_, T, Hkv, D, P, kv_dtype, max_pages=40, num_pages=None):
     x = x * torch.where(torch.rand(x.shape, generator=g) < 0.02, 1e-5, 1.0)
     k_new = x.to(torch.bfloat16)
     v_new = (-x * 0.5).to(torch.bfloat16)
-    k_new.view(-1)[5] = float("nan")
-    dt = torch.uint8 if kv_dtype == W.KV_FP8_E4M3 else torch.int16
-    shape = (num_pages, Hkv, P, D)
+    nv = kv_dtype == W.KV_NVFP4
+    if not nv:  # NVFP4 leaves the codes of NaN inputs unspecified
+        k_new.view(-1)[5] = float("nan")
+    else:  # blocks of zeros (scale 0) and of one large value among tiny ones
+        k_new.view(-1, 16)[3] = 0.0
+        v_new.view(-1, 16)[5] = 1e-6
+        v_new.view(-1, 16)[5, 7] = 3.0
+    dt = torch.uint8 if kv_dtype != W.KV_BF16 else torch.int16
+    shape = (num_pages, Hkv, P, D // 2 if nv else D)
     k_pages = torch.randint(-100, 100, shape, generator=g).to(dt)
     v_pages = torch.randint(-100, 100, shape, generator=g).to(dt)
     if dt == torch.int16:
         k_pages, v_pages = k_pages.view(torch.bfloat16), v_pages.view(torch.bfloat16)
-    return dict(k_new=k_new, v_new=v_new, page_table=page_table, kv_lens=kv_lens,
-                k_pages=k_pages, v_pages=v_pages, P=P, kv_dtype=kv_dtype)
+    c = dict(k_new=k_new, v_new=v_new, page_table=page_table, kv_lens=kv_lens,
+             k_pages=k_pages, v_pages=v_pages, P=P, kv_dtype=kv_dtype)
+    if nv:
+        sshape = (num_pages, Hkv, P, D // 16)
+        c["k_scales"] = torch.randint(0, 255, sshape, generator=g).to(torch.uint8)
+        c["v_scales"] = torch.randint(0, 255, sshape, generator=g).to(torch.uint8)
+    return c
 
 
 def _run_both(c, kv_scale=0.0123):
+    """The library's append and the oracle's on the same pools: returns the
+    library's pools, the oracle's, and the device error word (NVFP4 pools
+    come with their block-scale pools: (codes, scales) pairs)."""
     d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in c.items()}
     kp, vp = d["k_pages"].clone(), d["v_pages"].clone()
+    nv = c["kv_dtype"] == W.KV_NVFP4
+    sc = {}
+    if nv:
+        sc = dict(k_scales=d["k_scales"].clone(), v_scales=d["v_scales"].clone())
     B.paged_kv_append(d["k_new"], d["v_new"], d["page_table"], d["kv_lens"], kp, vp,
-                      kv_scale=kv_scale)
+                      kv_scale=kv_scale, **sc)
     torch.cuda.synchronize()
     err = B.last_device_error()
-    ok, ov = orc.paged_kv_append(W.to_bits(c["k_new"]), W.to_bits(c["v_new"]),
-                                 c["page_table"].numpy(), c["kv_lens"].numpy(),
-                                 W.to_bits(c["k_pages"]), W.to_bits(c["v_pages"]),
-                                 page_size=c["P"], kv_dtype=c["kv_dtype"], kv_scale=kv_scale)
-    return W.to_bits(kp.cpu()), W.to_bits(vp.cpu()), ok, ov, err
+    res = orc.paged_kv_append(W.to_bits(c["k_new"]), W.to_bits(c["v_new"]),
+                              c["page_table"].numpy(), c["kv_lens"].numpy(),
+                              W.to_bits(c["k_pages"]), W.to_bits(c["v_pages"]),
+                              page_size=c["P"], kv_dtype=c["kv_dtype"], kv_scale=kv_scale,
+                              k_scales=c.get("k_scales"), v_scales=c.get("v_scales"))
+    gk, gv = W.to_bits(kp.cpu()), W.to_bits(vp.cpu())
+    if nv:
+        return ((gk, W.to_bits(sc["k_scales"].cpu())), (gv, W.to_bits(sc["v_scales"].cpu())),
+                (res[0], res[2]), (res[1], res[3]), err)
+    return gk, gv, res[0], res[1], err
 
 
-@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3], ids=["bf16", "fp8"])
+def _equal(a, b):
+    if isinstance(a, tuple):
+        return all(np.array_equal(x, y) for x, y in zip(a, b))
+    return np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3, W.KV_NVFP4],
+                         ids=["bf16", "fp8", "nvfp4"])
 @pytest.mark.parametrize("D,P,T", [(64, 8, 1), (128, 16, 4), (128, 128, 13), (256, 32, 2)])
 def test_append_bit_exact(kv_dtype, D, P, T):
     c = _case(100 + D + P + T, 5, T, 3, D, P, kv_dtype)
     gk, gv, ok, ov, err = _run_both(c)
     assert err == 0
-    assert np.array_equal(gk, ok) and np.array_equal(gv, ov)
+    assert _equal(gk, ok) and _equal(gv, ov)
+
+
+@pytest.mark.parametrize("kv_scale", [0.0123, 1.0, 2.0 ** -14, 37.5])
+def test_append_nvfp4_bit_exact_across_scales(kv_scale):
+    """Per-tensor scales that put the block scales in e4m3's subnormal,
+    normal and saturating ranges."""
+    c = _case(400, 6, 3, 2, 128, 16, W.KV_NVFP4)
+    c["k_new"] = (c["k_new"].float() * torch.logspace(-6, 6, 128)).to(torch.bfloat16)
+    gk, gv, ok, ov, err = _run_both(c, kv_scale=kv_scale)
+    assert err == 0
+    assert _equal(gk, ok) and _equal(gv, ov)
 
 
 def test_append_large_batch_bit_exact():
@@ -94,7 +135,8 @@ def test_append_bad_page_is_reported_and_not_written():
     assert np.array_equal(W.to_bits(vp.cpu())[own], ov[own])
 
 
-@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3], ids=["bf16", "fp8"])
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8_E4M3, W.KV_NVFP4],
+                         ids=["bf16", "fp8", "nvfp4"])
 def test_append_then_decode(kv_dtype):
     """Append a decode step's new token (the cache the oracle appends the same
     way), then decode over the longer cache: parity with the oracle."""
@@ -114,19 +156,30 @@ def test_append_then_decode(kv_dtype):
     g = torch.Generator().manual_seed(4)
     k_new = torch.randn((wl.batch, 1, wl.num_kv_heads, wl.head_dim), generator=g).to(torch.bfloat16)
     v_new = torch.randn((wl.batch, 1, wl.num_kv_heads, wl.head_dim), generator=g).to(torch.bfloat16)
-    ok, ov = orc.paged_kv_append(W.to_bits(k_new), W.to_bits(v_new), pt.numpy(),
-                                 inp["kv_lens"].numpy(), W.to_bits(inp["k_pages"]),
-                                 W.to_bits(inp["v_pages"]), page_size=P, kv_dtype=kv_dtype,
-                                 kv_scale=inp["kv_scale"])
+    nv = kv_dtype == W.KV_NVFP4
+    res = orc.paged_kv_append(W.to_bits(k_new), W.to_bits(v_new), pt.numpy(),
+                              inp["kv_lens"].numpy(), W.to_bits(inp["k_pages"]),
+                              W.to_bits(inp["v_pages"]), page_size=P, kv_dtype=kv_dtype,
+                              kv_scale=inp["kv_scale"],
+                              k_scales=None if not nv else W.to_bits(inp["k_scales"]),
+                              v_scales=None if not nv else W.to_bits(inp["v_scales"]))
     d = U.to_device(dict(inp, page_table=pt))
     kp, vp = d["k_pages"].clone(), d["v_pages"].clone()
+    sc = {}
+    if nv:
+        sc = dict(k_scales=d["k_scales"].clone(), v_scales=d["v_scales"].clone())
     B.paged_kv_append(k_new.cuda(), v_new.cuda(), d["page_table"], d["kv_lens"], kp, vp,
-                      kv_scale=inp["kv_scale"])
+                      kv_scale=inp["kv_scale"], **sc)
     torch.cuda.synchronize()
     assert B.last_device_error() == 0
-    assert np.array_equal(W.to_bits(kp.cpu()), ok) and np.array_equal(W.to_bits(vp.cpu()), ov)
+    assert np.array_equal(W.to_bits(kp.cpu()), res[0])
+    assert np.array_equal(W.to_bits(vp.cpu()), res[1])
     new_lens = inp["kv_lens"] + 1
     after = dict(inp, page_table=pt, kv_lens=new_lens, k_pages=kp.cpu(), v_pages=vp.cpu())
+    if nv:
+        assert np.array_equal(W.to_bits(sc["k_scales"].cpu()), res[2])
+        assert np.array_equal(W.to_bits(sc["v_scales"].cpu()), res[3])
+        after.update(k_scales=sc["k_scales"].cpu(), v_scales=sc["v_scales"].cpu())
     ref_out, ref_lse = U.run_oracle(after)
     out, lse, _ = U.run_cuda(after)
     U.assert_parity(out, lse, ref_out, ref_lse, kv_dtype, "append then decode")

@@ -1,6 +1,6 @@
 """GPU parity: the CUDA library (through the C ABI) against the fp64 oracle on
-the same seeded inputs. Element by element on small and mid sizes spanning
-many tiles with ragged tails; sampled sequences at the full workload sizes."""
+the same seeded inputs, element by element: small and mid sizes spanning
+many tiles with ragged tails, and every row of the full workload sizes."""
 
 import zlib
 
@@ -14,7 +14,7 @@ from tests import gpu_util as U
 
 pytestmark = pytest.mark.gpu
 
-BF16, FP8 = W.KV_BF16, W.KV_FP8_E4M3
+BF16, FP8, NV = W.KV_BF16, W.KV_FP8_E4M3, W.KV_NVFP4
 BR = W.CAUSAL_BOTTOM_RIGHT
 
 
@@ -79,6 +79,18 @@ CASES = [
     # the bf16 tensor-core path (4 packed rows) on the same kind of scores
     wl("tc_bf16_peaked_g4", batch=2, num_q_heads=16, num_kv_heads=4, head_dim=128,
        page_size=16, scale=0.25, peaked_frac=0.01, kv_lens=("fixed", [3000, 8000])),
+    # NVFP4 K/V (e2m1 codes + an e4m3 scale per 16 elements), NaN scales in
+    # the slots no row may read
+    wl("nvfp4_headline_shape", batch=3, num_q_heads=32, num_kv_heads=8, head_dim=128,
+       page_size=16, kv_dtype=NV, kv_lens=("fixed", [1000, 517, 33]), extra_pages=3),
+    wl("nvfp4_verify_window", batch=3, q_len=4, num_q_heads=64, num_kv_heads=8,
+       head_dim=128, page_size=128, kv_dtype=NV, causal_offset=BR, window=512,
+       kv_lens=("fixed", [100, 700, 1500]), poison_invisible=True),
+    wl("nvfp4_d64_p8_gqa4", batch=2, num_q_heads=8, num_kv_heads=2, head_dim=64, page_size=8,
+       kv_dtype=NV, kv_lens=("fixed", [77, 300]), extra_pages=2),
+    wl("nvfp4_d256_p32_q2_window_peaked", batch=2, q_len=2, num_q_heads=4, num_kv_heads=2,
+       head_dim=256, page_size=32, kv_dtype=NV, causal_offset=BR, window=100, scale=0.25,
+       peaked_frac=0.02, kv_lens=("fixed", [700, 129]), poison_invisible=True, route="dense"),
 ]
 
 
@@ -117,19 +129,21 @@ def test_parity_forced_kernel(lib, case, splits, kernel):
     U.assert_parity(out, lse, ref_out, ref_lse, case.kv_dtype, f"{case.name}/{kernel}/s={splits}")
 
 
-@pytest.mark.parametrize("case", [CASES[2], CASES[5], CASES[7]], ids=lambda w: w.name)
+@pytest.mark.parametrize("case", [CASES[2], CASES[5], CASES[7]] +
+                         [c for c in CASES if c.kv_dtype == NV][:2], ids=lambda w: w.name)
 def test_page_permutation_invariance(lib, case):
     inp = W.generate(case)
     out0, lse0, _ = U.run_cuda(inp)
     n = inp["k_pages"].shape[0]
     perm = torch.randperm(n, generator=torch.Generator().manual_seed(7))
-    k2 = torch.empty_like(inp["k_pages"])
-    v2 = torch.empty_like(inp["v_pages"])
-    k2[perm] = inp["k_pages"]
-    v2[perm] = inp["v_pages"]
+    moved = {}
+    for key in ("k_pages", "v_pages", "k_scales", "v_scales"):
+        if inp.get(key) is not None:
+            moved[key] = torch.empty_like(inp[key])
+            moved[key][perm] = inp[key]
     pt = inp["page_table"].to(torch.int64)
     pt2 = torch.where(pt >= 0, perm[pt.clamp(min=0)], pt).to(torch.int32)
-    out1, lse1, _ = U.run_cuda(dict(inp, k_pages=k2, v_pages=v2, page_table=pt2))
+    out1, lse1, _ = U.run_cuda(dict(inp, page_table=pt2, **moved))
     # the kernel's arithmetic depends only on logical token order
     assert np.array_equal(out0, out1) and np.array_equal(lse0, lse1)
 
@@ -210,28 +224,44 @@ def _full(name):
     return W.ALL[name]
 
 
-@pytest.mark.parametrize("name,seqs", [
-    (W.HEADLINE.name, [0, 57, 127]),
-    (W.FP8_VERIFY.name, [0, 1, 33, 63]),
-])
-def test_full_size_sampled(lib, name, seqs):
-    case = _full(name)
-    inp = W.generate(case, device="cuda")
-    out, lse, used = U.run_cuda(inp)
-    ref_out, ref_lse = U.run_oracle(inp, seqs=seqs)
-    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, case.kv_dtype, name)
-    assert np.isfinite(out).all()
-
-
-def test_full_size_headline_cuda_core_kernel(lib):
-    """The headline shape through the CUDA-core kernel (the planner picks the
-    tensor-core kernel there)."""
+def test_full_size_headline_every_row(lib):
+    """The headline workload (B=128, kv_len 8192, bf16) in the benchmark's
+    launch configuration, every row against the oracle (run on all host
+    cores); then the same input through the CUDA-core kernel."""
     case = W.HEADLINE
     inp = W.generate(case, device="cuda")
+    ref_out, ref_lse = U.run_oracle(inp)
+    out, lse, _ = U.run_cuda(inp)
+    U.assert_parity(out, lse, ref_out, ref_lse, BF16, f"{case.name}/full/auto")
+    assert np.isfinite(out).all()
     out, lse, _ = U.run_cuda(inp, flags=B.PDA_FLAG_CUDA_CORES)
-    seqs = [3, 64, 126]
-    ref_out, ref_lse = U.run_oracle(inp, seqs=seqs)
-    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, BF16, "headline/cuda_cores")
+    U.assert_parity(out, lse, ref_out, ref_lse, BF16, f"{case.name}/full/cuda_cores")
+
+
+def test_full_size_fp8_verify_every_row(lib):
+    """The FP8 verify workload (B=64, q_len 4, lognormal lengths, window 4096)
+    in the benchmark's launch configuration, every row against the oracle on
+    the same e4m3 bytes: the exact two-term Q path, then native FP8 QK against
+    the oracle run on the same quantised q."""
+    case = W.FP8_VERIFY
+    inp = W.generate(case, device="cuda")
+    ref_out, ref_lse = U.run_oracle(inp)
+    out, lse, _ = U.run_cuda(inp)
+    U.assert_parity(out, lse, ref_out, ref_lse, FP8, f"{case.name}/full/auto")
+    assert np.isfinite(out).all()
+    ref_out, ref_lse = U.run_oracle(inp, native_qk=True)
+    out, lse, _ = U.run_cuda(inp, flags=B.PDA_FLAG_NATIVE_FP8_QK)
+    U.assert_parity(out, lse, ref_out, ref_lse, FP8, f"{case.name}/full/native_qk")
+
+
+def test_full_size_nvfp4_headline_every_row(lib):
+    """The headline shape with an NVFP4 KV cache, every row against the
+    oracle on the same codes and block scales."""
+    case = W.NVFP4_HEADLINE
+    inp = W.generate(case, device="cuda")
+    ref_out, ref_lse = U.run_oracle(inp)
+    out, lse, _ = U.run_cuda(inp)
+    U.assert_parity(out, lse, ref_out, ref_lse, NV, f"{case.name}/full")
 
 
 @pytest.mark.parametrize("name", [W.VARLEN.name, W.LONGCTX.name])
@@ -304,7 +334,8 @@ def test_cuda_graph_replays(lib):
 
 
 SINK_CASES = [c for c in CASES if c.head_dim == 128][:3] + \
-    [c for c in CASES if c.name.startswith("tc_fp8")][:2] + [CASES[0]]
+    [c for c in CASES if c.name.startswith("tc_fp8")][:2] + [CASES[0]] + \
+    [c for c in CASES if c.kv_dtype == NV][:1]
 
 
 @pytest.mark.parametrize("case", SINK_CASES, ids=lambda w: w.name)
@@ -341,15 +372,6 @@ def test_parity_native_fp8_qk(lib, case, splits):
     flags = B.PDA_FLAG_TENSOR_CORES | B.PDA_FLAG_NATIVE_FP8_QK
     out, lse, _ = U.run_cuda(inp, num_splits=splits, flags=flags)
     U.assert_parity(out, lse, ref_out, ref_lse, FP8, f"{case.name}/native/s={splits}")
-
-
-def test_full_size_fp8_verify_native_qk(lib):
-    case = _full(W.FP8_VERIFY.name)
-    inp = W.generate(case, device="cuda")
-    out, lse, _ = U.run_cuda(inp, flags=B.PDA_FLAG_NATIVE_FP8_QK)
-    seqs = [0, 17, 63]
-    ref_out, ref_lse = U.run_oracle(inp, seqs=seqs, native_qk=True)
-    U.assert_parity(out[seqs], lse[seqs], ref_out, ref_lse, FP8, "fp8 verify native qk")
 
 
 def _visible_tiles(wl, L, tile=128):
