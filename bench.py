@@ -48,7 +48,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
+    ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL) + sorted(W.EXTRA))
     ap.add_argument("--splits", type=int, default=0, help="force a split count (0: planner)")
     ap.add_argument("--kernel", choices=["auto", "tensor_cores", "cuda_cores"], default="auto",
                     help="split kernel: the planner's choice, or force one")
@@ -200,10 +200,15 @@ def recorded_traffic(workload_name: str, kernel_name: str):
 
 
 def algorithmic_bytes(wl: W.Workload, kv_lens):
-    """K/V bytes of keys some row may see + Q (bf16) + O (fp32) + LSE (fp32)."""
-    elt = 2 if wl.kv_dtype == W.KV_BF16 else 1
+    """K/V bytes of keys some row may see + Q (bf16) + O (fp32) + LSE (fp32).
+    A key's K (or V) row is D * 2 bytes in bf16, D in e4m3, and D/2 bytes of
+    codes plus D/16 bytes of block scales in NVFP4."""
     vis = W.visible_token_count(wl, kv_lens)
-    kv = vis * wl.num_kv_heads * wl.head_dim * elt * 2
+    if wl.kv_dtype == W.KV_NVFP4:
+        row = wl.head_dim // 2 + wl.head_dim // 16
+    else:
+        row = wl.head_dim * (2 if wl.kv_dtype == W.KV_BF16 else 1)
+    kv = vis * wl.num_kv_heads * row * 2
     rows = wl.batch * wl.q_len * wl.num_q_heads
     return kv + rows * wl.head_dim * 2 + rows * wl.head_dim * 4 + rows * 4, kv
 
@@ -323,7 +328,7 @@ def run_reference(args, rank, world):
         return
     # Same shapes and distributions, fewer sequences: the steps cycle over
     # (sequence, kv head) units of the first few sequences.
-    wl = W.ALL[args.workload]
+    wl = {**W.ALL, **W.EXTRA}[args.workload]
     inp = W.generate(wl.with_(batch=min(wl.batch, 4)), device="cpu")
     wl = inp["workload"]
     order = [(b, g) for b in range(wl.batch) for g in range(wl.num_kv_heads)]
@@ -391,15 +396,17 @@ def prepare(wl, dev, rank, splits, flags):
         kv_scale=inp["kv_scale"], max_kv_len=max_len, num_splits=splits, flags=flags)
     kernel_name = B.KERNEL_NAMES.get(B.plan_kernel(params), "unknown")
     ws = torch.empty(max(B.workspace_bytes(params), 1), dtype=torch.uint8, device=dev)
-    pool_bytes = kp.numel() * kp.element_size() * 2
-    pools = [(kp, vp)]
+    ks, vs = inp.get("k_scales"), inp.get("v_scales")  # NVFP4 block-scale pools
+    pool_bytes = kp.numel() * kp.element_size() * 2 + (0 if ks is None else ks.numel() * 2)
+    pools = [(kp, vp, ks, vs)]
     flush = None
     if pool_bytes >= ROTATE_BELOW_BYTES:
         l2 = (f"no flush: the K/V pools ({pool_bytes / 1e9:.2f} GB) are more than 8x the "
               "L2 (126 MB)")
     elif pool_bytes >= ROTATE_MIN_POOL_BYTES:
         n = max(2, -(-ROTATE_BELOW_BYTES // pool_bytes))
-        pools += [(kp.clone(), vp.clone()) for _ in range(n - 1)]
+        pools += [(kp.clone(), vp.clone(), None if ks is None else ks.clone(),
+                   None if vs is None else vs.clone()) for _ in range(n - 1)]
         l2 = (f"rotating {n} copies of the K/V pools ({pool_bytes / 1e9:.3f} GB each): "
               f"step i reads copy i mod {n}, so a copy returns after "
               f"{(n - 1) * pool_bytes / 1e9:.2f} GB of other K/V")
@@ -412,11 +419,11 @@ def prepare(wl, dev, rank, splits, flags):
 
 
 def call(ctx, i=0):
-    kp, vp = ctx["pools"][i % len(ctx["pools"])]
+    kp, vp, ks, vs = ctx["pools"][i % len(ctx["pools"])]
     inp = ctx["inp"]
     return B.paged_decode_attn(inp["q"], kp, vp, inp["page_table"], inp["kv_lens"],
                                out=ctx["out"], lse=ctx["lse"], workspace=ctx["ws"],
-                               **ctx["kw"])[2]
+                               k_scales=ks, v_scales=vs, **ctx["kw"])[2]
 
 
 def time_steps(ctx, steps, warmup, world, local):
@@ -551,7 +558,8 @@ def workload_entry(ctx, args, world, local, peak, probe_gbs, fused_merge, with_c
         "steps": args.steps, "warmup": args.warmup,
         "batch": wl.batch, "q_len": wl.q_len, "num_q_heads": wl.num_q_heads,
         "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "page_size": wl.page_size,
-        "kv_dtype": {W.KV_BF16: "bf16", W.KV_FP8_E4M3: "fp8_e4m3"}.get(wl.kv_dtype, wl.kv_dtype),
+        "kv_dtype": {W.KV_BF16: "bf16", W.KV_FP8_E4M3: "fp8_e4m3", W.KV_NVFP4: "nvfp4"}.get(
+            wl.kv_dtype, wl.kv_dtype),
         "l2": ctx["l2"],
         "timing": t["timing"],
         "launched": t["launched"],
@@ -568,7 +576,7 @@ def run_ours(args, rank, world, local):
     if not torch.cuda.is_available():
         raise RuntimeError("bench.py needs a CUDA device (the library has no CPU path)")
     B.load()
-    wl = W.ALL[args.workload]
+    wl = {**W.ALL, **W.EXTRA}[args.workload]
     if args.batch:
         wl = wl.with_(batch=args.batch, name=f"{wl.name}_batch{args.batch}")
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -632,7 +640,8 @@ def run_ours(args, rank, world, local):
             dq.copy_(hq, non_blocking=True)
             dpt.copy_(hpt, non_blocking=True)
             dkl.copy_(hkl, non_blocking=True)
-            B.paged_decode_attn(dq, kp, vp, dpt, dkl, out=out, lse=lse, workspace=ws, **kw)
+            B.paged_decode_attn(dq, kp, vp, dpt, dkl, out=out, lse=lse, workspace=ws,
+                                k_scales=inp.get("k_scales"), v_scales=inp.get("v_scales"), **kw)
             hout.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
 
@@ -661,21 +670,23 @@ def run_ours(args, rank, world, local):
     kv_append = None
     if not args.no_extras:
         kv_append = {}
-        elt = 2 if wl.kv_dtype == W.KV_BF16 else 1
+        # bytes per element written: bf16 2, e4m3 1, NVFP4 1/2 + 1/16 of a scale
+        elt = {W.KV_BF16: 2, W.KV_FP8_E4M3: 1, W.KV_NVFP4: 0.5625}[wl.kv_dtype]
         for T in (1, 64):
             if int(kl.min().item()) < T:
                 continue
             kn = torch.randn((wl.batch, T, wl.num_kv_heads, wl.head_dim), device=dev).to(torch.bfloat16)
             vn = torch.randn_like(kn)
             base = (kl - T).contiguous()
+            sc = dict(k_scales=inp.get("k_scales"), v_scales=inp.get("v_scales"))
             for _ in range(3):
-                B.paged_kv_append(kn, vn, pt, base, kp, vp, kv_scale=inp["kv_scale"])
+                B.paged_kv_append(kn, vn, pt, base, kp, vp, kv_scale=inp["kv_scale"], **sc)
             # 50 appends in one CUDA graph: device time, not Python call rate
             n_app = 50
             ga = torch.cuda.CUDAGraph()
             with torch.cuda.graph(ga):
                 for _ in range(n_app):
-                    B.paged_kv_append(kn, vn, pt, base, kp, vp, kv_scale=inp["kv_scale"])
+                    B.paged_kv_append(kn, vn, pt, base, kp, vp, kv_scale=inp["kv_scale"], **sc)
             ga.replay()
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a0.record(stream)
@@ -701,7 +712,7 @@ def run_ours(args, rank, world, local):
     if not (args.no_workloads or args.batch):
         workloads = {}
         with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
-        for name, other in W.ALL.items():
+        for name, other in list(W.ALL.items()) + list(W.EXTRA.items()):
             if name == wl.name:
                 entry = {
                     "ms_per_step": elapsed_ms / args.steps, "tokens_per_s": value,
@@ -728,6 +739,8 @@ def run_ours(args, rank, world, local):
                 octx = prepare(other, dev, rank, args.splits, flags)
                 entry = workload_entry(octx, args, world, local, peak, probe_gbs,
                                        args.fused_merge, with_cpu)
+                if name in W.EXTRA:
+                    entry["extra"] = "a KV dtype beyond the five workloads (the headline's shape)"
                 del octx
                 torch.cuda.empty_cache()
             workloads[name] = entry

@@ -52,10 +52,13 @@ def test_bench_line_carries_the_contract_fields():
     assert set(wls) == {"tiny_b2_gqa4_d64_p16", "varlen_b32_hq32_hkv8_d128_p64_l512to4096",
                         "b128_hq32_hkv8_d128_p16_l8192_bf16",
                         "longctx_b4_hq16_hkv4_d256_p128_l32768_peaked",
-                        "fp8_verify_b64_q4_hq64_hkv8_d128_p128_w4096"}
+                        "fp8_verify_b64_q4_hq64_hkv8_d128_p128_w4096",
+                        "nvfp4_b128_hq32_hkv8_d128_p16_l8192"}
+    assert wls["nvfp4_b128_hq32_hkv8_d128_p16_l8192"]["extra"]
+    assert wls["nvfp4_b128_hq32_hkv8_d128_p16_l8192"]["kv_dtype"] == "nvfp4"
     for name, e in wls.items():
         for k in ("ms_per_step", "tokens_per_s", "gb_s", "frac_of_copy", "frac_of_8tbs_spec",
-                  "kernel", "splits", "l2", "clocks", "avg_launch_ms",
+                  "kernel", "splits", "l2", "clocks", "avg_launch_ms", "timing", "launched",
                   "algorithmic_bytes_per_step", "cpu_baseline"):
             assert k in e, (name, k)
         assert e["gb_s"] == pytest.approx(
@@ -65,10 +68,13 @@ def test_bench_line_carries_the_contract_fields():
             e["batch"] * e["q_len"] / (e["ms_per_step"] / 1e3), rel=1e-6)
         assert e["cpu_baseline"]["kind"] == "oracle" and e["cpu_baseline"]["value"] > 0
         if name.startswith("tiny"):
-            assert e["l2"].startswith("flushed")
-        elif name.startswith("b128"):
-            assert e["l2"].startswith("no flush")
+            assert e["l2"].startswith("flushed") and e["timing"] == "host-launched"
         else:
-            assert e["l2"].startswith("rotating")
+            assert e["timing"].startswith("one CUDA graph")
+            if name.startswith("b128") or name.startswith("nvfp4"):
+                assert e["l2"].startswith("no flush")
+            else:
+                assert e["l2"].startswith("rotating")
+        assert e["launched"]["ms_per_step"] > 0
     top = wls[cfg["workload"]]
     assert top["top_level"] and top["ms_per_step"] == d["ms_per_step"]
