@@ -758,7 +758,8 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if wl.kv_dtype == W.KV_BF16 else "fp8_e4m3 kv, bf16 q, fp32 accumulate",
+        "dtype": {W.KV_BF16: "bf16", W.KV_FP8_E4M3: "fp8_e4m3 kv, bf16 q, fp32 accumulate",
+                  W.KV_NVFP4: "nvfp4 kv, bf16 q, fp32 accumulate"}[wl.kv_dtype],
         "data": "synthetic",
         "config": {
             "workload": wl.name, "batch": wl.batch, "q_len": wl.q_len,

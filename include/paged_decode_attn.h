@@ -329,9 +329,11 @@ PDA_API pda_status paged_kv_append(const void* k_new, const void* v_new,
  * variant and the tensor-core head-packing variant):
  *   PDA_KERNEL_SPLIT_TMA  tensor-core kernel (2D TMA tiles of 128 tokens,
  *                         tcgen05 MMAs with TMEM accumulators): head_dim 128
- *                         with bf16 K/V and at most 8 packed rows per kv head
- *                         (G * q_len), or FP8 K/V and more than 8; any
- *                         head_dim-128 case with PDA_FLAG_TENSOR_CORES;
+ *                         with bf16 or NVFP4 K/V and at most 8 packed rows
+ *                         per kv head (G * q_len; NVFP4 tiles are decoded
+ *                         exactly to f16 in shared memory), or FP8 K/V and
+ *                         more than 8; any head_dim-128 case with
+ *                         PDA_FLAG_TENSOR_CORES;
  *   PDA_KERNEL_SPLIT_FMA  CUDA-core kernel (warp-shuffle FMAs, cp.async.bulk
  *                         page copies): everything else, and every case with
  *                         PDA_FLAG_CUDA_CORES.

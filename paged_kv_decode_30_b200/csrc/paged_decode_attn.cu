@@ -95,9 +95,10 @@ bool pool_rows_fit(const pda_params* p) {
 // The flags force either kernel.
 bool use_tensor_cores(const pda_params* p, int M) {
   if (p->head_dim != 128 || p->page_size < 8 || !pool_rows_fit(p)) return false;
-  if (p->kv_dtype == PDA_KV_NVFP4) return false;  // the CUDA-core kernel decodes NVFP4
   if (p->flags & PDA_FLAG_CUDA_CORES) return false;
   if (p->flags & PDA_FLAG_TENSOR_CORES) return true;
+  // FP8: dense contractions with 16 or 32 rows; bf16 and NVFP4 (decoded to
+  // f16 tiles in shared memory): the 16-bit path with up to 8 rows
   return p->kv_dtype == PDA_KV_FP8_E4M3 ? M > 8 : M <= 8;
 }
 
@@ -136,7 +137,7 @@ Plan make_plan(const pda_params* p) {
     if (p->kv_dtype == PDA_KV_FP8_E4M3)
       pl.mt = pl.M <= 16 ? 16 : 32;  // rows per CTA; MMA N = 2 * rows for S^T
     else
-      pl.mt = pl.M <= 4 ? 4 : 8;     // bf16: N = 16 holds P^T hi and lo rows
+      pl.mt = pl.M <= 4 ? 4 : 8;     // 16-bit: N = 16 holds P^T hi and lo rows
     pl.tw = 128;                   // tokens per tile (MMA M)
     pl.tiles_per_cta_iter = 128;
   } else {

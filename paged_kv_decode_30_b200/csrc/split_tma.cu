@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <cstring>
 #include <mutex>
 
 #include "split_tma.cuh"
@@ -62,7 +63,7 @@ cudaError_t launch_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const Split
     __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
   }
   // prologue: block 0 (counters, queue order), FP8 one block per Q image
-  const long long q_blocks = KV ? (long long)a.B * a.Hkv * a.row_tiles : 0;
+  const long long q_blocks = KV == 1 ? (long long)a.B * a.Hkv * a.row_tiles : 0;
   if (q_blocks >= INT_MAX) return cudaErrorInvalidValue;
   split_tma_prologue<KV, NT, QN><<<dim3((unsigned)(1 + q_blocks)), 256, 0, stream>>>(a);
   e = cudaGetLastError();
@@ -89,6 +90,15 @@ cudaError_t launch_split_tma(int kv, int nt, bool native_qk, const void* k_pages
   const int elt = kv == 0 ? 2 : 1;
   const int box_rows = a.page_size < 128 ? a.page_size : 128;
   alignas(64) CUtensorMap mk, mv;
+  if (kv == 2) {  // NVFP4 tiles come by bulk copies: the maps are not read
+    std::memset(&mk, 0, sizeof(mk));
+    std::memset(&mv, 0, sizeof(mv));
+    switch (nt) {
+      case 4: return launch_cfg<2, 4>(mk, mv, a, grid, stream, pdl);
+      case 8: return launch_cfg<2, 8>(mk, mv, a, grid, stream, pdl);
+      default: return cudaErrorNotSupported;
+    }
+  }
   if (!make_pool_map(&mk, k_pages, rows, elt, box_rows) ||
       !make_pool_map(&mv, v_pages, rows, elt, box_rows))
     return cudaErrorInvalidValue;

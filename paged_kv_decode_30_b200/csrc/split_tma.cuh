@@ -71,9 +71,14 @@ struct ItemDesc {
 // QN (FP8 only): "native FP8 QK", Q enters the MMA as one e4m3 term per
 // element (q * 2^e rounded to nearest even, per-row power-of-two 2^e)
 // instead of the exact two-term split, so S^T has NT columns, not 2 NT.
+// KV: 0 bf16, 1 e4m3, 2 NVFP4. NVFP4 tiles arrive raw (codes and block
+// scales, by bulk copies) and converter warps decode them exactly into f16
+// tiles laid out as the TMA writes bf16 ones, so from the stages on the
+// NVFP4 path is the 16-bit path with f16 operands.
 template <int KV, int NT, bool QN = false>
 struct TmaCfg {
-  static constexpr bool BF16 = KV == 0;
+  static constexpr bool NV = KV == 2;
+  static constexpr bool BF16 = KV == 0 || NV;  // 16-bit operands (bf16; f16 for NVFP4)
   static constexpr bool QN_ = QN;
   static constexpr int D = 128;
   static constexpr int TILE = 128;
@@ -85,7 +90,14 @@ struct TmaCfg {
   // columns 16k .. 16k + 7 (hi term of rows 8k .. 8k + 7) and 16k + 8 ..
   // 16k + 15 (lo term), so a thread reads its rows' terms in one load.
   static constexpr int N2 = BF16 ? 16 : 2 * NT;
-  static constexpr int STAGES = BF16 ? 3 : 5;
+  static constexpr int STAGES = NV ? 2 : (BF16 ? 3 : 5);
+  // NVFP4: a ring of raw tiles, each K codes, K block scales, V codes and V
+  // scales of 128 tokens, that the converter warps decode into the stages
+  static constexpr int RAW_STAGES = NV ? 3 : 0;
+  static constexpr int RAW_C = TILE * D / 2;   // e2m1 codes of one K (or V) tile
+  static constexpr int RAW_S = TILE * D / 16;  // their e4m3 block scales
+  static constexpr int RAW_STAGE = 2 * (RAW_C + RAW_S);
+  static constexpr int CONV0 = 8, CONV_WARPS = NV ? 4 : 0;  // converter warps 8-11
   static constexpr int KT = TILE * D * ELT;      // bytes of one K (or V) tile
   static constexpr int STAGE = 2 * KT;           // K then V
   static constexpr int HALF = TILE * 128;        // one 128-byte column of SW128 atoms
@@ -107,7 +119,7 @@ struct TmaCfg {
   static constexpr int SOFT_H = BF16 ? 1 : NT / 8;  // row groups
   static constexpr int RH = NT / SOFT_H;             // rows per softmax thread
   static constexpr int SOFT_THREADS = 128 * SOFT_H;
-  static constexpr int WARPS = 8 + 4 * (SOFT_H - 1);
+  static constexpr int WARPS = 8 + 4 * (SOFT_H - 1) + CONV_WARPS;
   static constexpr int THREADS = WARPS * 32;
   // work-queue depths
   static constexpr int DSLOTS = 4;                 // item descriptors in flight
@@ -128,7 +140,8 @@ struct TmaCfg {
   static constexpr int SLOT = SL_SINK + 32 * 4;
   // shared memory map (1024-aligned where swizzled)
   static constexpr int OFF_STAGE = 0;
-  static constexpr int OFF_Q = OFF_STAGE + STAGES * STAGE;
+  static constexpr int OFF_RAW = OFF_STAGE + STAGES * STAGE;
+  static constexpr int OFF_Q = OFF_RAW + RAW_STAGES * RAW_STAGE;
   static constexpr int OFF_P = OFF_Q + 2 * Q_BUF;
   static constexpr int P_BUF = ((P_BYTES + 1023) / 1024) * 1024;
   // FP8: a 32-token x 128 tile of e4m3 ones, the A operand of the MMAs that
@@ -144,8 +157,9 @@ struct TmaCfg {
   static constexpr int OFF_PIDS = OFF_DESC + DSLOTS * (int)sizeof(Desc);
   static constexpr int OFF_BAR = OFF_PIDS + PID_SLOTS * 16 * 4;
   // full[S], empty[S], s_full[2], p_ready[2], o_full[2], o_free[2],
-  // desc_full[4], desc_free[4], q_ready[2], st_free[2], q_free[2]
-  static constexpr int NUM_BARS = 2 * STAGES + 8 + 2 * DSLOTS + 6;
+  // desc_full[4], desc_free[4], q_ready[2], st_free[2], q_free[2],
+  // NVFP4: raw_full[R], raw_empty[R], k_full[S]
+  static constexpr int NUM_BARS = 2 * STAGES + 8 + 2 * DSLOTS + 6 + 2 * RAW_STAGES + (NV ? STAGES : 0);
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
   // [0] abort, [1] tiles done, [4 + k] merge flag of row group k
   static constexpr int OFF_FLAGS = OFF_TMEM_SLOT + 8;
@@ -159,6 +173,7 @@ struct TmaCfg {
   static_assert(!(BF16 && QN), "native QK is an FP8 option");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
   static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 && OFF_ONES % 1024 == 0, "alignment");
+  static_assert(!NV || SOFT_H == 1, "NVFP4: one softmax group, converter warps at 8-11");
   static_assert(BF16 || RH == 8, "FP8: 8 rows per softmax thread");
   static_assert(sizeof(Desc) % 16 == 0 && OFF_DESC % 16 == 0 && OFF_SLOTS % 16 == 0, "alignment");
 };
@@ -173,10 +188,11 @@ __host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N) {
 __host__ __device__ constexpr uint32_t umma_idesc_e4m3_mn(int M, int N) {
   return umma_idesc_e4m3(M, N) | (1u << 15) | (1u << 16);
 }
-// kind::f16 with bf16 A and B.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// kind::f16 with bf16 A and B (f16 A and B when f16 is set), fp32 D.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn, bool b_mn,
+                                                       bool f16 = false) {
+  return (1u << 4) | (f16 ? 0u : (1u << 7) | (1u << 10)) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -232,6 +248,19 @@ __device__ __forceinline__ uint32_t e4m3_split2(float p0, float p1) {
   return (uint32_t)h | ((uint32_t)lo << 16);
 }
 
+// Eight e2m1 codes (one word, element 2k in the low nibble of byte k) ->
+// four f16 pairs (exact), element 2k in the low half of h[k].
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t* h) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code & 0xFF), __NV_E4M3);
   return __half2float(*reinterpret_cast<const __half*>(&h));
@@ -284,6 +313,10 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
   uint64_t* q_ready = desc_free + C::DSLOTS;   // [2] Q operand + per-row state written
   uint64_t* st_free = q_ready + 2;             // [2] per-row state of an item released
   uint64_t* q_free = st_free + 2;              // [2] S^T MMAs of an item done (its Q reusable)
+  uint64_t* raw_full = q_free + 2;             // NVFP4 [R] raw tile landed
+  uint64_t* raw_empty = raw_full + C::RAW_STAGES;  // NVFP4 [R] raw tile decoded
+  uint64_t* k_full = raw_empty + C::RAW_STAGES;    // NVFP4 [S] f16 K of the stage written
+                                                   // (full[]: its V too)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   volatile int* tiles_done = abort_flag + 1;  // tiles the softmax warps have finished
   volatile int* merge_flag = abort_flag + 4;  // [row group]
@@ -293,9 +326,17 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
 
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // TMA: the producer's arrive and the copies' bytes; NVFP4: every
+      // converter thread's arrive once the f16 tile is written
+      mbar_init(&full[s], C::NV ? 32 * C::CONV_WARPS : 1);
       mbar_init(&empty[s], 1);  // the O^T MMAs of the tile are done
     }
+    for (int s = 0; s < C::RAW_STAGES; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], 32 * C::CONV_WARPS);
+    }
+    if constexpr (C::NV)
+      for (int s = 0; s < C::STAGES; ++s) mbar_init(&k_full[s], 32 * C::CONV_WARPS);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_ready[i], C::SOFT_THREADS);
@@ -474,6 +515,33 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
                 a.q + ((long long)(b * a.Lq + qi) * a.Hq + h) * C::D + jj * 8));
           }
         }
+        if constexpr (C::NV) {
+          // NVFP4: the MMAs take f16, so each bf16 q row enters as f16 of
+          // q * 2^e, 2^e the power of two that puts the row's max |q| in
+          // [2^14, 2^15): exact for every element within 2^28 of the row's
+          // max (smaller ones round in f16's subnormal range); the score
+          // scale of the row carries 2^-e. The 16 lanes of a row are adjacent.
+#pragma unroll
+          for (int k = 0; k < QREG; ++k) {
+            const int c = lane + 32 * k, n = c >> 4, jj = c & 15;
+            float f[8];
+            bf16x8_to_f32(qv[k], f);
+            float mx = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+            const int e2 = mx > 0.f ? 14 - ilogbf(mx) : 0;
+            uint32_t hw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __half2 h = __floats2half2_rn(ldexpf(f[2 * e], e2), ldexpf(f[2 * e + 1], e2));
+              hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            qv[k] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            if (jj == 0 && n < NT) cs[n] = ldexpf(a.qk_scale_log2, -e2);
+          }
+        }
 #pragma unroll
         for (int k = 0; k < QREG; ++k) {
           const int c = lane + 32 * k, n = c >> 4, jj = c & 15;
@@ -481,7 +549,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             *reinterpret_cast<uint4*>(qbuf + (jj >> 3) * C::Q_HALF + (n >> 3) * 1024 +
                                       (n & 7) * 128 + (((jj & 7) ^ (n & 7)) << 4)) = qv[k];
         }
-        if (lane < NT) cs[lane] = a.qk_scale_log2;
+        if (!C::NV && lane < NT) cs[lane] = a.qk_scale_log2;
       } else {
         // the prologue kernel's image of this (b, kv head, row tile): one bulk
         // copy, counted on q_ready next to the 32 lanes' arrivals below
@@ -554,7 +622,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     // so "tile n's group is complete" is cp.async.wait_group PA-1).
     int32_t* sm_pids = reinterpret_cast<int32_t*>(smem + C::OFF_PIDS);
     const uint32_t sbase = smem_addr(smem);
-    if (lane == 0) {
+    if (!C::NV && lane == 0) {  // (NVFP4 copies take no tensor map)
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmk) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmv) : "memory");
     }
@@ -601,29 +669,62 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           }
           asm volatile("cp.async.commit_group;" ::: "memory");
         }
-        const int st = g % C::STAGES;
-        ok = !*abort_flag;
-        if (ok && g >= C::STAGES) ok = mbar_wait(&empty[st], ((g / C::STAGES) - 1) & 1, a.err);
-        if (!__all_sync(FULL, ok)) {
-          ok = false;
-          break;
-        }
         const int tok0 = (kfirst + n) * C::TILE;
         const int nseg = nseg_of(n);
-        const uint32_t seg_bytes = (uint32_t)seg_rows * 128u * (C::BF16 ? 2u : 1u);
-        const uint32_t kdst = sbase + C::OFF_STAGE + st * C::STAGE;
-        const uint32_t vdst = kdst + C::KT;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2u * seg_bytes * (uint32_t)nseg);
-        __syncwarp();  // the transaction count is set before any copy completes
-        if (lane < nseg) {  // lane s copies segment s: a tile's copies go out together
-          const int row = (pid * a.Hkv + kvh) * a.page_size +
-                          (a.page_size >= C::TILE ? (tok0 & (a.page_size - 1)) : 0);
-          const uint32_t off = (uint32_t)lane * seg_rows * 128u;
-          tma_load_2d(kdst + off, &tmk, 0, row, &full[st]);
-          tma_load_2d(vdst + off, &tmv, 0, row, &full[st]);
-          if constexpr (C::BF16) {  // second 64-element half of each row
-            tma_load_2d(kdst + C::HALF + off, &tmk, 64, row, &full[st]);
-            tma_load_2d(vdst + C::HALF + off, &tmv, 64, row, &full[st]);
+        if constexpr (C::NV) {
+          // raw NVFP4 tile: per page segment, its codes (64 bytes per token)
+          // and block scales (8 bytes per token) of K and V, four bulk copies
+          // into raw slot g % RAW_STAGES, decoded by the converter warps
+          const int rs = g % C::RAW_STAGES;
+          ok = !*abort_flag;
+          if (ok && g >= C::RAW_STAGES)
+            ok = mbar_wait(&raw_empty[rs], ((g / C::RAW_STAGES) - 1) & 1, a.err);
+          if (!__all_sync(FULL, ok)) {
+            ok = false;
+            break;
+          }
+          uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_STAGE;
+          uint64_t* rb = &raw_full[rs];
+          if (lane == 0)
+            mbar_arrive_expect_tx(rb, 2u * (uint32_t)(nseg * seg_rows) * (uint32_t)(C::D / 2 + C::D / 16));
+          __syncwarp();  // the transaction count is set before any copy completes
+          if (lane < nseg) {
+            const long long row = (long long)(pid * a.Hkv + kvh) * a.page_size +
+                                  (a.page_size >= C::TILE ? (tok0 & (a.page_size - 1)) : 0);
+            const uint32_t cbytes = (uint32_t)seg_rows * (C::D / 2);
+            const uint32_t sbytes = (uint32_t)seg_rows * (C::D / 16);
+            uint8_t* kc = raw + lane * cbytes;
+            uint8_t* ks = raw + C::RAW_C + lane * sbytes;
+            uint8_t* vc = raw + C::RAW_C + C::RAW_S + lane * cbytes;
+            uint8_t* vs = raw + 2 * C::RAW_C + C::RAW_S + lane * sbytes;
+            bulk_g2s(kc, a.k_pages + row * (C::D / 2), cbytes, rb);
+            bulk_g2s(ks, a.k_scales + row * (C::D / 16), sbytes, rb);
+            bulk_g2s(vc, a.v_pages + row * (C::D / 2), cbytes, rb);
+            bulk_g2s(vs, a.v_scales + row * (C::D / 16), sbytes, rb);
+          }
+        } else {
+          const int st = g % C::STAGES;
+          ok = !*abort_flag;
+          if (ok && g >= C::STAGES) ok = mbar_wait(&empty[st], ((g / C::STAGES) - 1) & 1, a.err);
+          if (!__all_sync(FULL, ok)) {
+            ok = false;
+            break;
+          }
+          const uint32_t seg_bytes = (uint32_t)seg_rows * 128u * (C::BF16 ? 2u : 1u);
+          const uint32_t kdst = sbase + C::OFF_STAGE + st * C::STAGE;
+          const uint32_t vdst = kdst + C::KT;
+          if (lane == 0) mbar_arrive_expect_tx(&full[st], 2u * seg_bytes * (uint32_t)nseg);
+          __syncwarp();  // the transaction count is set before any copy completes
+          if (lane < nseg) {  // lane s copies segment s: a tile's copies go out together
+            const int row = (pid * a.Hkv + kvh) * a.page_size +
+                            (a.page_size >= C::TILE ? (tok0 & (a.page_size - 1)) : 0);
+            const uint32_t off = (uint32_t)lane * seg_rows * 128u;
+            tma_load_2d(kdst + off, &tmk, 0, row, &full[st]);
+            tma_load_2d(vdst + off, &tmv, 0, row, &full[st]);
+            if constexpr (C::BF16) {  // second 64-element half of each row
+              tma_load_2d(kdst + C::HALF + off, &tmk, 64, row, &full[st]);
+              tma_load_2d(vdst + C::HALF + off, &tmv, 64, row, &full[st]);
+            }
           }
         }
       }
@@ -633,8 +734,14 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       if (lane == 0) {
         *abort_flag = 1;
         // copies already issued land before the CTA's shared memory goes away
-        for (int n = max(0, g - C::STAGES); n < g; ++n)
-          mbar_wait(&full[n % C::STAGES], (n / C::STAGES) & 1, a.err, kWaitTimeoutCycles / 16);
+        if constexpr (C::NV) {
+          for (int n = max(0, g - C::RAW_STAGES); n < g; ++n)
+            mbar_wait(&raw_full[n % C::RAW_STAGES], (n / C::RAW_STAGES) & 1, a.err,
+                      kWaitTimeoutCycles / 16);
+        } else {
+          for (int n = max(0, g - C::STAGES); n < g; ++n)
+            mbar_wait(&full[n % C::STAGES], (n / C::STAGES) & 1, a.err, kWaitTimeoutCycles / 16);
+        }
       }
     }
     __syncwarp();
@@ -654,7 +761,8 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           ok = mbar_wait(&q_ready[j & 1], (j >> 1) & 1, a.err);  // Q of item j
           for (int n = 0; ok && n < ntiles; ++n, ++g) {
             const int bb = g & 1;
-            ok = !*abort_flag && mbar_wait(&full[g % C::STAGES], (g / C::STAGES) & 1, a.err);
+            ok = !*abort_flag && mbar_wait(C::NV ? &k_full[g % C::STAGES] : &full[g % C::STAGES],
+                                           (g / C::STAGES) & 1, a.err);  // K of tile g
             if (ok && g >= 2) ok = mbar_wait(&p_ready[bb], ((g - 2) >> 1) & 1, a.err);
             if (!ok) break;
             tmem_fence_after();
@@ -662,7 +770,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             const uint32_t qa = sbase + C::OFF_Q + (j & 1) * C::Q_BUF;
             const uint32_t dt = tmem + C::COL_S + bb * C::N1;
             if constexpr (C::BF16) {
-              constexpr uint32_t idesc = umma_idesc_bf16(128, C::N1, false, false);
+              constexpr uint32_t idesc = umma_idesc_bf16(128, C::N1, false, false, C::NV);
 #pragma unroll
               for (int s = 0; s < C::D / 16; ++s)
                 umma_f16(dt, umma_desc(ka + (s >> 2) * C::HALF + (s & 3) * 32, 16, 1024, kSw128),
@@ -686,13 +794,15 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           for (int n = 0; ok && n < ntiles; ++n, ++g) {
             const int bb = g & 1;
             ok = !*abort_flag && mbar_wait(&p_ready[bb], (g >> 1) & 1, a.err);
+            // NVFP4: the f16 V of the stage (written after its K)
+            if (C::NV && ok) ok = mbar_wait(&full[g % C::STAGES], (g / C::STAGES) & 1, a.err);
             if (!ok) break;
             tmem_fence_after();
             const uint32_t pa = sbase + C::OFF_P + bb * C::P_BUF;
             const uint32_t dt = tmem + C::COL_O + (j & 1) * C::N2;
             const uint32_t va = sbase + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT;
             if constexpr (C::BF16) {
-              constexpr uint32_t idesc = umma_idesc_bf16(128, C::N2, true, true);
+              constexpr uint32_t idesc = umma_idesc_bf16(128, C::N2, true, true, C::NV);
 #pragma unroll
               for (int s = 0; s < C::TILE / 16; ++s)
                 umma_f16(dt, umma_desc(va + s * 2048, C::HALF, 1024, kSw128),
@@ -730,6 +840,92 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
       }
     }
     __syncwarp();
+  } else if (C::NV && warp >= C::CONV0 && warp < C::CONV0 + C::CONV_WARPS) {
+    // ======================= NVFP4 converters (warps 8-11) ====================
+    // Tile g: raw slot g % RAW_STAGES -> f16 stage g % STAGES, K then V. A
+    // task is 32 consecutive elements of one token (16 code bytes, two
+    // 16-element blocks): task k = token k / 4, quarter k % 4, so a warp's
+    // loads of one instruction cover 512 contiguous bytes. Each byte of two
+    // e2m1 codes becomes an f16 pair (cvt.rn.f16x2.e2m1x2), times its
+    // block's scale (an f16 pair from cvt.rn.f16x2.e4m3x2): exact, since an
+    // e2m1 x e4m3 product has 5 significant bits and lies in f16's normal
+    // range. The f16 rows go to the 128B-swizzled layout the TMA writes for
+    // bf16 (two 64-element halves of 8-row atoms), which the MMAs read.
+    const int ct = tid - C::CONV0 * 32;  // 0 .. 32 * CONV_WARPS - 1
+    constexpr int CT = 32 * C::CONV_WARPS;
+    int g = 0;
+    bool ok = true;
+    for (int j = 0; ok; ++j) {
+      ok = !*abort_flag && mbar_wait(&desc_full[j & (C::DSLOTS - 1)], (j / C::DSLOTS) & 1, a.err);
+      if (!__all_sync(FULL, ok)) {
+        ok = false;
+        break;
+      }
+      const Desc& d = descs[j & (C::DSLOTS - 1)];
+      if (d.b < 0) break;
+      const int ntiles = d.ntiles;
+      for (int n = 0; n < ntiles; ++n, ++g) {
+        const int rs = g % C::RAW_STAGES, st = g % C::STAGES;
+        const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_STAGE;
+        uint8_t* stage = smem + C::OFF_STAGE + st * C::STAGE;
+        ok = !*abort_flag && mbar_wait(&raw_full[rs], (g / C::RAW_STAGES) & 1, a.err);
+        if (!__all_sync(FULL, ok)) {
+          ok = false;
+          break;
+        }
+#pragma unroll 1
+        for (int pool = 0; ok && pool < 2; ++pool) {
+          // K of the stage is free once the S^T MMAs of tile g - STAGES are
+          // done, V once its O^T MMAs are (S^T(g) cannot complete before this
+          // K is written, so the s_full phase waited for is the right one)
+          if (g >= C::STAGES)
+            ok = pool == 0 ? mbar_wait(&s_full[(g - C::STAGES) & 1], ((g - C::STAGES) >> 1) & 1, a.err)
+                           : mbar_wait(&empty[st], ((g / C::STAGES) - 1) & 1, a.err);
+          if (!__all_sync(FULL, ok)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* codes = raw + pool * (C::RAW_C + C::RAW_S);
+          const uint8_t* scales = codes + C::RAW_C;
+          uint8_t* dst = stage + pool * C::KT;
+#pragma unroll
+          for (int k = ct; k < C::TILE * 4; k += CT) {
+            const int t = k >> 2, qq = k & 3;
+            const uint4 c = *reinterpret_cast<const uint4*>(codes + t * (C::D / 2) + qq * 16);
+            const uint32_t sc2 = *reinterpret_cast<const uint16_t*>(scales + t * (C::D / 16) + 2 * qq);
+            const __half2_raw sr = __nv_cvt_fp8x2_to_halfraw2(
+                static_cast<__nv_fp8x2_storage_t>(sc2), __NV_E4M3);
+            const __half2 s2 = *reinterpret_cast<const __half2*>(&sr);
+            const __half2 sa = __low2half2(s2), sb = __high2half2(s2);
+            const uint32_t w[4] = {c.x, c.y, c.z, c.w};  // block 2qq: w[0..1]; 2qq + 1: w[2..3]
+            uint32_t o[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              e2m1x8_to_f16x8(w[q], o + 4 * q);
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&o[4 * q + b]), q < 2 ? sa : sb);
+                o[4 * q + b] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+            }
+            // elements 32 qq .. 32 qq + 31: half qq / 2, chunks 4 (qq & 1) .. + 3
+            uint8_t* row = dst + (qq >> 1) * C::HALF + (t >> 3) * 1024 + (t & 7) * 128;
+            const int cb = (qq & 1) * 4;
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              *reinterpret_cast<uint4*>(row + (((cb + k4) ^ (t & 7)) << 4)) =
+                  make_uint4(o[4 * k4], o[4 * k4 + 1], o[4 * k4 + 2], o[4 * k4 + 3]);
+          }
+          fence_proxy_async_smem();  // read by the tensor core (and, once both
+                                     // pools are done, the raw slot is refilled)
+          mbar_arrive(pool == 0 ? &k_full[st] : &full[st]);
+        }
+        if (!ok) break;
+        mbar_arrive(&raw_empty[rs]);
+      }
+      if (!ok) break;
+    }
+    if (!ok) *abort_flag = 1;
   } else if ((warp >= C::SOFT0 && warp < C::SOFT0 + 4) ||
              (C::SOFT_H > 1 && warp >= C::SOFTX && warp < C::SOFTX + 4 * (C::SOFT_H - 1))) {
     // ======================= softmax ==========================================
@@ -1037,6 +1233,11 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
           // jt; group 0 only. Chunks in rotated order: the 8 rows of a
           // 1 KB swizzle atom hit 8 different bank groups.
           if (grp == 0 && (jt < lo_u || jt >= hi_u)) {
+            // NVFP4: the f16 V of the stage is written after its K, so wait
+            // for it before zeroing rows (no later write can come: the next
+            // tile into this stage waits for this one's O^T MMAs)
+            if (C::NV && !mbar_wait(&full[g % C::STAGES], (g / C::STAGES) & 1, a.err))
+              acc_ok = false;
             uint8_t* vrow = smem + C::OFF_STAGE + (g % C::STAGES) * C::STAGE + C::KT + i * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -1155,13 +1356,22 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
         const int pswz = C::P_ROW == 64 ? ((i & 7) >> 1) & 3 : ((i & 7) >> 2) & 1;
         if constexpr (C::BF16) {
           // columns 0..NT-1: bf16(p); NT..2NT-1: bf16(p - bf16(p)); rest stay 0
+          // (NVFP4: the same two terms in f16, the MMAs' operand type)
           uint32_t w[NT];  // NT/2 words of hi, then NT/2 of lo
 #pragma unroll
           for (int r = 0; r < NT; r += 2) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(p[r], p[r + 1]);
-            const float2 hf = __bfloat1622float2(h);
-            w[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
-            w[NT / 2 + r / 2] = pack_bf16x2(p[r] - hf.x, p[r + 1] - hf.y);
+            if constexpr (C::NV) {
+              const __half2 h = __floats2half2_rn(p[r], p[r + 1]);
+              const float2 hf = __half22float2(h);
+              const __half2 l = __floats2half2_rn(p[r] - hf.x, p[r + 1] - hf.y);
+              w[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
+              w[NT / 2 + r / 2] = *reinterpret_cast<const uint32_t*>(&l);
+            } else {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(p[r], p[r + 1]);
+              const float2 hf = __bfloat1622float2(h);
+              w[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
+              w[NT / 2 + r / 2] = pack_bf16x2(p[r] - hf.x, p[r + 1] - hf.y);
+            }
           }
           if constexpr (NT == 8) {
             *reinterpret_cast<uint4*>(sp + ((0 ^ pswz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);

@@ -291,6 +291,11 @@ def test_nvfp4_needs_aligned_scale_pools(lib):
     a = B.PdaAppendParams(4, 1, 8, 128, 16, 8, 64, B.PDA_KV_NVFP4, 0.01, None, None)
     st = lib.paged_kv_append(ok, ok, ok, ok, ctypes.byref(a), ok, ok, None)
     assert st == 1
-    # the planner keeps NVFP4 on the CUDA-core kernel, whatever the flags
-    p = headline_params(kv_dtype=B.PDA_KV_NVFP4, kv_scale=0.01, flags=B.PDA_FLAG_TENSOR_CORES)
+    # head_dim 128 with at most 8 packed rows: the tensor-core kernel (NVFP4
+    # decoded to f16 tiles); other head dims, or the flag: the CUDA-core one
+    p = headline_params(kv_dtype=B.PDA_KV_NVFP4, kv_scale=0.01)
+    assert B.plan_kernel(p) == B.PDA_KERNEL_SPLIT_TMA
+    p = headline_params(kv_dtype=B.PDA_KV_NVFP4, kv_scale=0.01, flags=B.PDA_FLAG_CUDA_CORES)
+    assert B.plan_kernel(p) == B.PDA_KERNEL_SPLIT_FMA
+    p = headline_params(kv_dtype=B.PDA_KV_NVFP4, kv_scale=0.01, head_dim=64)
     assert B.plan_kernel(p) == B.PDA_KERNEL_SPLIT_FMA
