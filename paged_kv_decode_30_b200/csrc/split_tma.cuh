@@ -46,6 +46,10 @@
 //    An item's epilogue (normalise, store O and the LSE, or the split's
 //    partials; with the fused merge, the split that arrives last for its
 //    rows merges them all) runs after the next item's first tile.
+//  * NVFP4 K/V: the producer bulk-copies raw tiles (e2m1 codes and e4m3
+//    block scales) into a ring of their own, and warps 8-11 (converters)
+//    decode them exactly into f16 tiles in the stages' layout; the MMAs then
+//    run kind::f16 with f16 operands (q as f16 of q * 2^e per row).
 //  * Every wait is bounded; group exits go through bar.red.and.
 #pragma once
 
