@@ -91,6 +91,14 @@ CASES = [
     wl("nvfp4_d256_p32_q2_window_peaked", batch=2, q_len=2, num_q_heads=4, num_kv_heads=2,
        head_dim=256, page_size=32, kv_dtype=NV, causal_offset=BR, window=100, scale=0.25,
        peaked_frac=0.02, kv_lens=("fixed", [700, 129]), poison_invisible=True, route="dense"),
+    # NVFP4 on the tensor-core kernel: whole-tile pages, 8 packed rows,
+    # peaked scores; then windowed verify rows with empty and 1-key sequences
+    wl("nvfp4_tc_p256_g8_peaked", batch=3, num_q_heads=16, num_kv_heads=2, head_dim=128,
+       page_size=256, kv_dtype=NV, scale=0.25, peaked_frac=0.01,
+       kv_lens=("fixed", [3000, 257, 4096]), route="dense"),
+    wl("nvfp4_tc_p64_q2_window_empty", batch=4, q_len=2, num_q_heads=8, num_kv_heads=4,
+       head_dim=128, page_size=64, kv_dtype=NV, causal_offset=BR, window=300,
+       kv_lens=("fixed", [0, 1, 900, 2000]), poison_invisible=True, extra_pages=2),
 ]
 
 
