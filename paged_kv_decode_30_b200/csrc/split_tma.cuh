@@ -845,91 +845,93 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
     }
     __syncwarp();
   } else if (C::NV && warp >= C::CONV0 && warp < C::CONV0 + C::CONV_WARPS) {
-    // ======================= NVFP4 converters (warps 8-11) ====================
-    // Tile g: raw slot g % RAW_STAGES -> f16 stage g % STAGES, K then V. A
-    // task is 32 consecutive elements of one token (16 code bytes, two
-    // 16-element blocks): task k = token k / 4, quarter k % 4, so a warp's
-    // loads of one instruction cover 512 contiguous bytes. Each byte of two
-    // e2m1 codes becomes an f16 pair (cvt.rn.f16x2.e2m1x2), times its
-    // block's scale (an f16 pair from cvt.rn.f16x2.e4m3x2): exact, since an
-    // e2m1 x e4m3 product has 5 significant bits and lies in f16's normal
-    // range. The f16 rows go to the 128B-swizzled layout the TMA writes for
-    // bf16 (two 64-element halves of 8-row atoms), which the MMAs read.
-    const int ct = tid - C::CONV0 * 32;  // 0 .. 32 * CONV_WARPS - 1
-    constexpr int CT = 32 * C::CONV_WARPS;
-    int g = 0;
-    bool ok = true;
-    for (int j = 0; ok; ++j) {
-      ok = !*abort_flag && mbar_wait(&desc_full[j & (C::DSLOTS - 1)], (j / C::DSLOTS) & 1, a.err);
-      if (!__all_sync(FULL, ok)) {
-        ok = false;
-        break;
-      }
-      const Desc& d = descs[j & (C::DSLOTS - 1)];
-      if (d.b < 0) break;
-      const int ntiles = d.ntiles;
-      for (int n = 0; n < ntiles; ++n, ++g) {
-        const int rs = g % C::RAW_STAGES, st = g % C::STAGES;
-        const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_STAGE;
-        uint8_t* stage = smem + C::OFF_STAGE + st * C::STAGE;
-        ok = !*abort_flag && mbar_wait(&raw_full[rs], (g / C::RAW_STAGES) & 1, a.err);
+    if constexpr (C::NV) {  // (compiled for NVFP4 only)
+      // ======================= NVFP4 converters (warps 8-11) ====================
+      // Tile g: raw slot g % RAW_STAGES -> f16 stage g % STAGES, K then V. A
+      // task is 32 consecutive elements of one token (16 code bytes, two
+      // 16-element blocks): task k = token k / 4, quarter k % 4, so a warp's
+      // loads of one instruction cover 512 contiguous bytes. Each byte of two
+      // e2m1 codes becomes an f16 pair (cvt.rn.f16x2.e2m1x2), times its
+      // block's scale (an f16 pair from cvt.rn.f16x2.e4m3x2): exact, since an
+      // e2m1 x e4m3 product has 5 significant bits and lies in f16's normal
+      // range. The f16 rows go to the 128B-swizzled layout the TMA writes for
+      // bf16 (two 64-element halves of 8-row atoms), which the MMAs read.
+      const int ct = tid - C::CONV0 * 32;  // 0 .. 32 * CONV_WARPS - 1
+      constexpr int CT = 32 * C::CONV_WARPS;
+      int g = 0;
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
+        ok = !*abort_flag && mbar_wait(&desc_full[j & (C::DSLOTS - 1)], (j / C::DSLOTS) & 1, a.err);
         if (!__all_sync(FULL, ok)) {
           ok = false;
           break;
         }
-#pragma unroll 1
-        for (int pool = 0; ok && pool < 2; ++pool) {
-          // K of the stage is free once the S^T MMAs of tile g - STAGES are
-          // done, V once its O^T MMAs are (S^T(g) cannot complete before this
-          // K is written, so the s_full phase waited for is the right one)
-          if (g >= C::STAGES)
-            ok = pool == 0 ? mbar_wait(&s_full[(g - C::STAGES) & 1], ((g - C::STAGES) >> 1) & 1, a.err)
-                           : mbar_wait(&empty[st], ((g / C::STAGES) - 1) & 1, a.err);
+        const Desc& d = descs[j & (C::DSLOTS - 1)];
+        if (d.b < 0) break;
+        const int ntiles = d.ntiles;
+        for (int n = 0; n < ntiles; ++n, ++g) {
+          const int rs = g % C::RAW_STAGES, st = g % C::STAGES;
+          const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_STAGE;
+          uint8_t* stage = smem + C::OFF_STAGE + st * C::STAGE;
+          ok = !*abort_flag && mbar_wait(&raw_full[rs], (g / C::RAW_STAGES) & 1, a.err);
           if (!__all_sync(FULL, ok)) {
             ok = false;
             break;
           }
-          const uint8_t* codes = raw + pool * (C::RAW_C + C::RAW_S);
-          const uint8_t* scales = codes + C::RAW_C;
-          uint8_t* dst = stage + pool * C::KT;
-#pragma unroll
-          for (int k = ct; k < C::TILE * 4; k += CT) {
-            const int t = k >> 2, qq = k & 3;
-            const uint4 c = *reinterpret_cast<const uint4*>(codes + t * (C::D / 2) + qq * 16);
-            const uint32_t sc2 = *reinterpret_cast<const uint16_t*>(scales + t * (C::D / 16) + 2 * qq);
-            const __half2_raw sr = __nv_cvt_fp8x2_to_halfraw2(
-                static_cast<__nv_fp8x2_storage_t>(sc2), __NV_E4M3);
-            const __half2 s2 = *reinterpret_cast<const __half2*>(&sr);
-            const __half2 sa = __low2half2(s2), sb = __high2half2(s2);
-            const uint32_t w[4] = {c.x, c.y, c.z, c.w};  // block 2qq: w[0..1]; 2qq + 1: w[2..3]
-            uint32_t o[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              e2m1x8_to_f16x8(w[q], o + 4 * q);
-#pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                const __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&o[4 * q + b]), q < 2 ? sa : sb);
-                o[4 * q + b] = *reinterpret_cast<const uint32_t*>(&h);
-              }
+  #pragma unroll 1
+          for (int pool = 0; ok && pool < 2; ++pool) {
+            // K of the stage is free once the S^T MMAs of tile g - STAGES are
+            // done, V once its O^T MMAs are (S^T(g) cannot complete before this
+            // K is written, so the s_full phase waited for is the right one)
+            if (g >= C::STAGES)
+              ok = pool == 0 ? mbar_wait(&s_full[(g - C::STAGES) & 1], ((g - C::STAGES) >> 1) & 1, a.err)
+                             : mbar_wait(&empty[st], ((g / C::STAGES) - 1) & 1, a.err);
+            if (!__all_sync(FULL, ok)) {
+              ok = false;
+              break;
             }
-            // elements 32 qq .. 32 qq + 31: half qq / 2, chunks 4 (qq & 1) .. + 3
-            uint8_t* row = dst + (qq >> 1) * C::HALF + (t >> 3) * 1024 + (t & 7) * 128;
-            const int cb = (qq & 1) * 4;
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-              *reinterpret_cast<uint4*>(row + (((cb + k4) ^ (t & 7)) << 4)) =
-                  make_uint4(o[4 * k4], o[4 * k4 + 1], o[4 * k4 + 2], o[4 * k4 + 3]);
+            const uint8_t* codes = raw + pool * (C::RAW_C + C::RAW_S);
+            const uint8_t* scales = codes + C::RAW_C;
+            uint8_t* dst = stage + pool * C::KT;
+  #pragma unroll
+            for (int k = ct; k < C::TILE * 4; k += CT) {
+              const int t = k >> 2, qq = k & 3;
+              const uint4 c = *reinterpret_cast<const uint4*>(codes + t * (C::D / 2) + qq * 16);
+              const uint32_t sc2 = *reinterpret_cast<const uint16_t*>(scales + t * (C::D / 16) + 2 * qq);
+              const __half2_raw sr = __nv_cvt_fp8x2_to_halfraw2(
+                  static_cast<__nv_fp8x2_storage_t>(sc2), __NV_E4M3);
+              const __half2 s2 = *reinterpret_cast<const __half2*>(&sr);
+              const __half2 sa = __low2half2(s2), sb = __high2half2(s2);
+              const uint32_t w[4] = {c.x, c.y, c.z, c.w};  // block 2qq: w[0..1]; 2qq + 1: w[2..3]
+              uint32_t o[16];
+  #pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                e2m1x8_to_f16x8(w[q], o + 4 * q);
+  #pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  const __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&o[4 * q + b]), q < 2 ? sa : sb);
+                  o[4 * q + b] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+              }
+              // elements 32 qq .. 32 qq + 31: half qq / 2, chunks 4 (qq & 1) .. + 3
+              uint8_t* row = dst + (qq >> 1) * C::HALF + (t >> 3) * 1024 + (t & 7) * 128;
+              const int cb = (qq & 1) * 4;
+  #pragma unroll
+              for (int k4 = 0; k4 < 4; ++k4)
+                *reinterpret_cast<uint4*>(row + (((cb + k4) ^ (t & 7)) << 4)) =
+                    make_uint4(o[4 * k4], o[4 * k4 + 1], o[4 * k4 + 2], o[4 * k4 + 3]);
+            }
+            fence_proxy_async_smem();  // read by the tensor core (and, once both
+                                       // pools are done, the raw slot is refilled)
+            mbar_arrive(pool == 0 ? &k_full[st] : &full[st]);
           }
-          fence_proxy_async_smem();  // read by the tensor core (and, once both
-                                     // pools are done, the raw slot is refilled)
-          mbar_arrive(pool == 0 ? &k_full[st] : &full[st]);
+          if (!ok) break;
+          mbar_arrive(&raw_empty[rs]);
         }
         if (!ok) break;
-        mbar_arrive(&raw_empty[rs]);
       }
-      if (!ok) break;
+      if (!ok) *abort_flag = 1;
     }
-    if (!ok) *abort_flag = 1;
   } else if ((warp >= C::SOFT0 && warp < C::SOFT0 + 4) ||
              (C::SOFT_H > 1 && warp >= C::SOFTX && warp < C::SOFTX + 4 * (C::SOFT_H - 1))) {
     // ======================= softmax ==========================================
