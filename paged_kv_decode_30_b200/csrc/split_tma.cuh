@@ -878,7 +878,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             ok = false;
             break;
           }
-  #pragma unroll 1
+#pragma unroll 1
           for (int pool = 0; ok && pool < 2; ++pool) {
             // K of the stage is free once the S^T MMAs of tile g - STAGES are
             // done, V once its O^T MMAs are (S^T(g) cannot complete before this
@@ -893,7 +893,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
             const uint8_t* codes = raw + pool * (C::RAW_C + C::RAW_S);
             const uint8_t* scales = codes + C::RAW_C;
             uint8_t* dst = stage + pool * C::KT;
-  #pragma unroll
+#pragma unroll
             for (int k = ct; k < C::TILE * 4; k += CT) {
               const int t = k >> 2, qq = k & 3;
               const uint4 c = *reinterpret_cast<const uint4*>(codes + t * (C::D / 2) + qq * 16);
@@ -904,10 +904,10 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
               const __half2 sa = __low2half2(s2), sb = __high2half2(s2);
               const uint32_t w[4] = {c.x, c.y, c.z, c.w};  // block 2qq: w[0..1]; 2qq + 1: w[2..3]
               uint32_t o[16];
-  #pragma unroll
+#pragma unroll
               for (int q = 0; q < 4; ++q) {
                 e2m1x8_to_f16x8(w[q], o + 4 * q);
-  #pragma unroll
+#pragma unroll
                 for (int b = 0; b < 4; ++b) {
                   const __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&o[4 * q + b]), q < 2 ? sa : sb);
                   o[4 * q + b] = *reinterpret_cast<const uint32_t*>(&h);
@@ -916,7 +916,7 @@ __global__ void __launch_bounds__(TmaCfg<KV, NT, QN>::THREADS, 1)
               // elements 32 qq .. 32 qq + 31: half qq / 2, chunks 4 (qq & 1) .. + 3
               uint8_t* row = dst + (qq >> 1) * C::HALF + (t >> 3) * 1024 + (t & 7) * 128;
               const int cb = (qq & 1) * 4;
-  #pragma unroll
+#pragma unroll
               for (int k4 = 0; k4 < 4; ++k4)
                 *reinterpret_cast<uint4*>(row + (((cb + k4) ^ (t & 7)) << 4)) =
                     make_uint4(o[4 * k4], o[4 * k4 + 1], o[4 * k4 + 2], o[4 * k4 + 3]);
