@@ -116,6 +116,14 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _own_copy(a, dtype) -> np.ndarray:
+    """A C-contiguous copy of `a` as `dtype` (array-likes that offer
+    .numpy(), such as CPU tensors, are read through it)."""
+    if not isinstance(a, np.ndarray) and hasattr(a, "numpy"):
+        a = a.numpy()
+    return np.array(a, dtype=dtype, copy=True, order="C")
+
+
 def bf16_to_double(bits: int, lib=None) -> float:
     return (lib or load()).oracle_bf16_to_double(int(bits))
 
@@ -226,16 +234,16 @@ def paged_kv_append(k_new_bits, v_new_bits, page_table, kv_lens, k_pages, v_page
     k_new_bits = np.ascontiguousarray(k_new_bits, dtype=np.uint16)
     v_new_bits = np.ascontiguousarray(v_new_bits, dtype=np.uint16)
     kdt = np.uint16 if kv_dtype == ORACLE_KV_BF16 else np.uint8
-    kp = np.array(k_pages, dtype=kdt, copy=True, order="C")
-    vp = np.array(v_pages, dtype=kdt, copy=True, order="C")
+    kp = _own_copy(k_pages, kdt)
+    vp = _own_copy(v_pages, kdt)
     page_table = np.ascontiguousarray(page_table, dtype=np.int32)
     kv_lens = np.ascontiguousarray(kv_lens, dtype=np.int32)
     B, num_new, Hkv, D = k_new_bits.shape
     nv = kv_dtype == ORACLE_KV_NVFP4
     ks = vs = None
     if nv:
-        ks = np.array(k_scales, dtype=np.uint8, copy=True, order="C")
-        vs = np.array(v_scales, dtype=np.uint8, copy=True, order="C")
+        ks = _own_copy(k_scales, np.uint8)
+        vs = _own_copy(v_scales, np.uint8)
     rc = lib.oracle_paged_kv_append(
         _ptr(k_new_bits), _ptr(v_new_bits), _ptr(page_table), _ptr(kv_lens), B, num_new,
         Hkv, D, page_size, page_table.shape[1], kp.shape[0], int(kv_dtype), float(kv_scale),
