@@ -50,6 +50,13 @@ def test_fp8_bytes_are_one_byte_per_element():
     assert total == kv + rows * (128 * 2 + 128 * 4 + 4)
 
 
+def test_nvfp4_bytes_are_codes_plus_block_scales():
+    # a K (or V) row of 128 elements: 64 bytes of e2m1 codes + 8 e4m3 scales
+    total, kv = bench.algorithmic_bytes(W.NVFP4_HEADLINE, [8192] * 128)
+    assert kv == 128 * 8192 * 8 * (64 + 8) * 2 == 1_207_959_552
+    assert total == kv + 1_048_576 + 2_097_152 + 16_384 == 1_211_121_664
+
+
 @pytest.mark.parametrize("causal_offset,window,q_len", list(itertools.product(
     [W.CAUSAL_OFF, W.CAUSAL_BOTTOM_RIGHT, 0, 5, 40], [0, 1, 7, 33], [1, 4, 8])))
 def test_visible_count_matches_the_rule(causal_offset, window, q_len):
